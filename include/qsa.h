@@ -1,0 +1,144 @@
+/*
+ * qsa.h -- C ABI of the B200 (sm_100a) Top-K-selected sparse attention library
+ * used for QSA prefill (libqsa.so).
+ *
+ * Source of the operation: the article "Qwen4-Exp QSA comes to Huawei's Ascend:
+ * inside SGLang's opt-in CANN prefill PR" (orcarouter.ai blog).
+ *   - section "What the pull request actually adds": attention over already-rotated
+ *     Q and K, scale * Q K^T, softmax, times V (the packed-embedding paragraph); the
+ *     original head-dim-256 scale is kept; unordered physical slots with -1 padding;
+ *     fully masked rows keep the zero-output convention; supported local head shapes
+ *     (16,2), (24,2), (12,1), (6,1), (3,1); BF16 with head dimension 256.
+ *   - section "Nine tests that passed, and a speed number that did not come from this
+ *     branch": unordered physical slots at widths 1/63/64/65/2051, default and explicit
+ *     scales, fully masked rows, zero selection width, non-contiguous tensors, an FP32
+ *     CPU reference from the same BF16 inputs, and the long-prefill case
+ *     (7,810 queries x 2,051 selected slots over a 65,536-slot cache).
+ *   - section "Why QSA is the awkward part, in numbers": sparse block size 1 (one
+ *     selected slot is one token) and the untouched selected-token interface.
+ *
+ * What one call computes.  Let G = Hq / Hkv.  For every query row t in [0, Tq) and
+ * every query head h in [0, Hq), with KV head j = floor(h / G):
+ *
+ *   V_t   = { slot_idx[t, w] : 0 <= w < width[t], slot_idx[t, w] != -1 }   (a multiset)
+ *   s_i   = scale * sum_d q[t, h, d] * k_cache[V_t[i], j, d]
+ *   p_i   = exp(s_i - max_i s_i),  l = sum_i p_i
+ *   out[t, h, :] = sum_i p_i * v_cache[V_t[i], j, :] / l,      or exactly +0 if V_t is empty.
+ *
+ * The order of the slots in a row does not matter; -1 may appear anywhere inside the
+ * first width[t] entries and is skipped; entries at w >= width[t] are never read.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are bf16 (q, k_cache, v_cache, out) or int32 (slot_idx, width) in
+ *     DEVICE memory, owned by the caller.  The library allocates nothing, never
+ *     synchronises the stream or the device, and only enqueues work on `stream`.
+ *   - Strides are in ELEMENTS of the tensor's own type.  The innermost (d) stride is 1.
+ *     q is [Tq, Hq, D], k_cache / v_cache are [S, Hkv, D], out is [Tq, Hq, D],
+ *     slot_idx is [Tq, W] (row stride idx_stride_t, column stride 1), width is [Tq]
+ *     contiguous.
+ *   - Only D == 256 and 1 <= G <= 16 are implemented (QSA_ERR_UNSUPPORTED otherwise).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).
+ */
+#ifndef QSA_H_
+#define QSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1, /* a NULL required pointer, a negative size, Hq % Hkv != 0,
+                              a misaligned base or stride, a NaN/Inf scale, too small a
+                              workspace for the requested split count                */
+  QSA_ERR_UNSUPPORTED = 2, /* D != 256, or G = Hq / Hkv outside 1..16                    */
+  QSA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than the plan requires          */
+  QSA_ERR_CUDA = 4         /* a CUDA runtime call or a kernel launch failed             */
+} qsa_status_t;
+
+/* Bits that the kernels OR into *err_word (device memory, optional). */
+#define QSA_ERRBIT_SLOT_RANGE 0x1u /* a slot index outside [-1, S) was seen; it was masked */
+#define QSA_ERRBIT_WIDTH_RANGE 0x2u /* a width[t] outside [0, W] was seen; it was clamped   */
+
+/* Largest number of selected positions one split processes (the per-split index list
+ * is staged whole in shared memory).  Wider selections are split automatically. */
+#define QSA_MAX_SLOTS_PER_SPLIT 2560
+
+/* Version of this ABI; bumped on any signature change. */
+int32_t qsa_abi_version(void);
+
+/*
+ * qsa_sparse_prefill_plan -- host-only planner (no CUDA call, no device access).
+ *
+ * Returns the number of W-splits `nsplit` that qsa_sparse_prefill will use for this
+ * shape and writes the matching workspace size in bytes to *workspace_bytes (may be
+ * NULL).  nsplit_request == 0 asks for the automatic choice for a device with
+ * `num_sms` multiprocessors; nsplit_request > 0 forces that count (it is raised to
+ * the minimum that keeps every split within QSA_MAX_SLOTS_PER_SPLIT positions and
+ * lowered to at most W).  With nsplit == 1 no workspace is needed (0 bytes).
+ * With nsplit > 1 the workspace holds fp32 partial outputs [nsplit, Tq, Hq, D] and
+ * base-2 log-sum-exp values [nsplit, Tq, Hq], each region 256-byte aligned.
+ * Returns a negative qsa_status_t value (e.g. -QSA_ERR_INVALID_ARG) when the shape
+ * itself is invalid or unsupported.
+ */
+int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W,
+                                int32_t num_sms, int32_t nsplit_request,
+                                size_t* workspace_bytes);
+
+/*
+ * qsa_sparse_prefill -- selected-slot sparse attention for one prefill batch.
+ *
+ * Arguments (all device pointers unless stated):
+ *   q            bf16 [Tq, Hq, D], strides (q_stride_t, q_stride_h, 1).  Already rotated.
+ *   k_cache      bf16 [S, Hkv, D], strides (k_stride_s, k_stride_h, 1).  Already rotated.
+ *   v_cache      bf16 [S, Hkv, D], strides (v_stride_s, v_stride_h, 1).
+ *   slot_idx     int32 [Tq, W], row stride idx_stride_t.  Unordered physical slots;
+ *                -1 = masked.  Any other value outside [0, S) is masked as well and sets
+ *                QSA_ERRBIT_SLOT_RANGE in *err_word.
+ *   width        int32 [Tq] selection width per row, or NULL meaning W for every row.
+ *                Values outside [0, W] are clamped and set QSA_ERRBIT_WIDTH_RANGE
+ *                (the host cannot see device values without a synchronisation).
+ *   Tq, Hq, Hkv, D, S, W   sizes; Tq == 0 is a no-op returning QSA_OK; W == 0 writes
+ *                exact zeros.
+ *   scale        multiplier of Q K^T (1/sqrt(256) = 1/16 keeps the original scale).
+ *   out          bf16 [Tq, Hq, D], strides (out_stride_t, out_stride_h, 1).  Written in
+ *                full (rows with no valid slot get +0.0).  Must not alias the inputs.
+ *   nsplit       0 = automatic (the planner's choice for the current device), else the
+ *                requested split count (adjusted exactly as qsa_sparse_prefill_plan does).
+ *   workspace    device scratch of at least the planned size (may be NULL when the plan
+ *                needs 0 bytes).  Contents on entry are irrelevant.
+ *   err_word     device uint32 that receives QSA_ERRBIT_* bits via atomic OR, or NULL.
+ *                The caller clears it; it is read back whenever the caller chooses.
+ *   stream       cudaStream_t on which all work is enqueued.
+ *
+ * Alignment: q, k_cache, v_cache and out must be 16-byte aligned and their t/h/s
+ * strides multiples of 8 elements (16 bytes); slot_idx and width 4-byte aligned.
+ * Errors are reported before any launch and leave `out` untouched.  The call is
+ * deterministic: the same inputs give bitwise the same `out` (inputs are read-only).
+ */
+qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                const int32_t* slot_idx, int64_t idx_stride_t,
+                                const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                int32_t D, int64_t S, int32_t W, float scale, void* out,
+                                int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
+                                void* workspace, size_t workspace_bytes, uint32_t* err_word,
+                                void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* qsa_status_string(qsa_status_t status);
+
+/* Detail of the most recent non-OK status returned on the calling host thread
+ * (static thread-local storage; "" if none). */
+const char* qsa_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_H_ */

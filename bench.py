@@ -1,0 +1,342 @@
+"""Benchmark of the sparse-prefill hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one full pass of the hot path (slot compaction, K/V gather, QK^T, online
+softmax, PV, epilogue; plus the LSE combine when the plan splits W) over the long
+prefill batch: Hq=16, Hkv=2, D=256, S=65,536 cache slots, Tq=7,810 query rows,
+W=2,051 distinct unordered slots per row (the long-prefill case of the article
+"Qwen4-Exp QSA comes to Huawei's Ascend: inside SGLang's opt-in CANN prefill PR",
+section "Nine tests that passed, ...").  Inputs are synthetic (N(0,1) bf16, uniform
+distinct slots) and resident in HBM before the timed region; L2 is flushed between
+steps by writing a 512 MiB buffer.  Multi-GPU runs are independent replicas (the path
+has no exchange step): every rank processes its own batch and the value is the total
+over ranks divided by the slowest rank's time.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle on a bounded
+sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+import torch
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+from top_sparse_attention_index_b200 import workloads as wl  # noqa: E402
+
+METRIC = "sparse prefill TFLOP/s & query-slot pairs/s, 7810q×2051 sel; % of roofline"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def work_counts(w: wl.Workload):
+    """Valid (t, slot) pairs and the algorithmic FLOPs / bytes of one pass."""
+    W = w.W
+    pos = torch.arange(W)[None, :]
+    wt = torch.full((w.Tq, 1), W) if w.width is None else w.width.to(torch.int64)[:, None]
+    ok = (pos < wt) & (w.slot_idx >= 0) & (w.slot_idx < w.S)
+    pairs = int(ok.sum())
+    D = w.q.shape[2]
+    flops = pairs * w.Hq * 4 * D                         # 2D (QK^T) + 2D (PV) per head
+    gathered = pairs * w.Hkv * 2 * D * 2                 # K and V rows, bf16
+    other = w.Tq * w.Hq * D * 2 * 2 + w.Tq * W * 4       # Q in, out, indices
+    return pairs, flops, gathered + other, gathered
+
+
+def measured_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        ids = [x.strip() for x in vis.split(",")] if vis else []
+        self.gpu_index = ids[gpu_index] if gpu_index < len(ids) else str(gpu_index)
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(w: wl.Workload, flops_per_row: float, target_s: float):
+    """The oracle as it stands on the host cores, on a bounded sample of query rows."""
+    import oracle
+    o = oracle.default()
+    probe = list(range(16))
+    t0 = time.perf_counter()
+    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0, rows=probe)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    n = int(min(w.Tq, max(64, len(probe) * target_s / dt)))
+    rows = list(range(n))
+    t0 = time.perf_counter()
+    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = flops_per_row * n  # every row of this workload has the same valid width
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": o.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"first {n} of {w.Tq} query rows of the same workload (all heads, all selected slots)"}
+
+
+def run_reference(args, rank):
+    """--impl reference: the CPU oracle, timed on the host, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    w = wl.long_prefill()
+    pairs, flops, _, _ = work_counts(w)
+    per_row = flops / w.Tq
+    o = oracle.default()
+    rows_per_step = 128
+    for s in range(args.warmup):
+        o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0,
+                  rows=list(range((s * rows_per_step) % w.Tq, (s * rows_per_step) % w.Tq + rows_per_step)))
+    times = []
+    for s in range(args.steps):
+        r0 = ((args.warmup + s) * rows_per_step) % (w.Tq - rows_per_step)
+        t0 = time.perf_counter()
+        o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0,
+                  rows=list(range(r0, r0 + rows_per_step)))
+        times.append(time.perf_counter() - t0)
+    sec = sum(times)
+    value = per_row * rows_per_step * args.steps / sec / 1e12
+    sample = f"{rows_per_step} consecutive query rows per step (of {w.Tq}), all heads and slots"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sec / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": 256, "S": w.S,
+                   "W": w.W, "valid_pairs": pairs, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": o.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    import top_sparse_attention_index_b200 as qsa
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    w = wl.long_prefill()
+    pairs, flops, alg_bytes, gathered = work_counts(w)
+    q, k, v, idx = (x.to(device) for x in (w.q, w.k_cache, w.v_cache, w.slot_idx))
+    out = torch.empty(w.Tq, w.Hq, 256, dtype=torch.bfloat16, device=device)
+    num_sms = torch.cuda.get_device_properties(device).multi_processor_count
+    nsplit, ws_bytes = qsa.qsa_sparse_prefill_plan(w.Tq, w.Hq, w.Hkv, 256, w.W, num_sms)
+    launches_per_step = 1 if nsplit == 1 else 2
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        qsa.sparse_prefill(q, k, v, idx, scale=1.0 / 16.0, out=out)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if dist is not None:
+        dist.barrier()
+    kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = torch.tensor([sum(kernel_ms)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    total_ms = float(total_ms.item())
+    ms_per_step = total_ms / args.steps
+
+    # end to end through the public API: pinned host inputs -> device -> kernel -> host
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hidx = (x.pin_memory() for x in (w.q, w.k_cache, w.v_cache, w.slot_idx))
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hidx))
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            idx.copy_(hidx, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e_steps = max(3, min(args.steps, 10))
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        es.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        ee.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([es.elapsed_time(ee) / e_steps], dtype=torch.float64, device=device)
+        if dist is not None:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * flops / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": float(e_ms.item()), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = measured_peaks()
+    t_s = ms_per_step * 1e-3
+    achieved = alg_bytes / t_s / 1e9
+    traffic = None
+    prof = ROOT / "profiles" / "traffic.json"
+    if prof.exists():
+        tj = json.loads(prof.read_text())
+        if tj.get("kernel_source_hash") == _kernel_hash():
+            traffic = tj.get("bytes_per_launch")
+    result = {
+        "metric": METRIC,
+        "value": world * flops / t_s / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": 256, "S": w.S,
+                   "W": w.W, "valid_pairs": pairs, "nsplit": nsplit,
+                   "l2": "flushed between steps (512 MiB write)", "parallelism": f"replicas x{world}"},
+        "pairs_per_s": world * pairs / t_s,
+        "pairs_x_hkv_per_s": world * pairs * w.Hkv / t_s,
+        "gathered_gb_per_s": gathered / t_s / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": alg_bytes},
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": clocks.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, flops / w.Tq, args.cpu_seconds)
+    print(json.dumps(result))
+
+
+def _kernel_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for p in sorted((ROOT / "top_sparse_attention_index_b200" / "csrc").glob("*")):
+        h.update(p.read_bytes())
+    return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    main()

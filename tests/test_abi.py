@@ -1,0 +1,162 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports every
+symbol include/qsa.h declares, the planner's choices, and argument validation that
+returns before any CUDA call."""
+from __future__ import annotations
+
+import ctypes
+import re
+import subprocess
+from pathlib import Path
+
+import pytest
+import torch
+
+import top_sparse_attention_index_b200 as qsa
+from top_sparse_attention_index_b200 import _binding, build_lib
+
+HEADER = Path(__file__).resolve().parent.parent / "include" / "qsa.h"
+
+
+def declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", HEADER.read_text(), flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(qsa_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return _binding.load_library()
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted(_binding.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", str(_binding.LIBRARY)],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (qsa_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_library_is_built_for_sm100a():
+    text = build_lib.NVCC_FLAGS
+    assert "arch=compute_100a,code=sm_100a" in text
+
+
+def test_status_strings(lib):
+    assert qsa.qsa_abi_version() == 1
+    for code, name in [(0, "QSA_OK"), (1, "QSA_ERR_INVALID_ARG"), (2, "QSA_ERR_UNSUPPORTED"),
+                       (3, "QSA_ERR_WORKSPACE"), (4, "QSA_ERR_CUDA")]:
+        assert qsa.qsa_status_string(code) == name
+
+
+@pytest.mark.parametrize("Tq,Hq,Hkv,W,expect", [
+    (7810, 16, 2, 2051, 1),       # long prefill: enough units, one split
+    (128, 16, 2, 64, 1),          # tiny: a 64-wide row is never split
+    (16384, 24, 2, 2051, 1),      # causal two-request
+    (4096, 6, 1, 2048, 1),        # max extent
+])
+def test_plan_without_split(lib, Tq, Hq, Hkv, W, expect):
+    n, ws = qsa.qsa_sparse_prefill_plan(Tq, Hq, Hkv, 256, W, 148)
+    assert n == expect and ws == 0
+
+
+def test_plan_splits_small_batches(lib):
+    n, ws = qsa.qsa_sparse_prefill_plan(257, 12, 1, 256, 2051, 148)
+    assert n > 1
+    assert ws >= n * 257 * 12 * 256 * 4 + n * 257 * 12 * 4
+    n1, _ = qsa.qsa_sparse_prefill_plan(1, 16, 2, 256, 2051, 148)
+    assert n1 == 16  # floor(2051 / 128): splits are never narrower than 128 positions
+    assert -(-2051 // n1) >= 128
+
+
+def test_plan_wide_rows_force_splits(lib):
+    n, _ = qsa.qsa_sparse_prefill_plan(100000, 16, 2, 256, 6000, 148)
+    assert n == 3  # ceil(6000 / 2560)
+    n, _ = qsa.qsa_sparse_prefill_plan(100000, 16, 2, 256, 6000, 148, 1)
+    assert n == 3  # a request below the minimum is raised
+    n, _ = qsa.qsa_sparse_prefill_plan(10, 16, 2, 256, 5, 148, 64)
+    assert n == 5  # ... and one above W lowered
+    n, ws = qsa.qsa_sparse_prefill_plan(10, 16, 2, 256, 0, 148)
+    assert n == 1 and ws == 0
+
+
+@pytest.mark.parametrize("shape,status", [
+    ((4, 16, 3, 256, 8), qsa.QSA_ERR_INVALID_ARG),   # Hq % Hkv
+    ((4, 16, 2, 128, 8), qsa.QSA_ERR_UNSUPPORTED),   # D != 256
+    ((4, 17, 1, 256, 8), qsa.QSA_ERR_UNSUPPORTED),   # G = 17
+    ((-1, 16, 2, 256, 8), qsa.QSA_ERR_INVALID_ARG),  # negative Tq
+    ((4, 16, 2, 256, -3), qsa.QSA_ERR_INVALID_ARG),  # negative W
+    ((4, 0, 2, 256, 8), qsa.QSA_ERR_INVALID_ARG),
+])
+def test_plan_rejects(lib, shape, status):
+    with pytest.raises(qsa.QSAError) as ei:
+        qsa.qsa_sparse_prefill_plan(*shape, 148)
+    assert ei.value.status == status
+
+
+def _call(**over):
+    """A raw ABI call with fake (never dereferenced) aligned pointers; every test below
+    makes exactly one argument invalid so the call returns before touching CUDA."""
+    a = dict(q=0x10000, q_stride_t=16 * 256, q_stride_h=256, k_cache=0x20000, k_stride_s=512,
+             k_stride_h=256, v_cache=0x30000, v_stride_s=512, v_stride_h=256, slot_idx=0x40000,
+             idx_stride_t=8, width=None, Tq=4, Hq=16, Hkv=2, D=256, S=100, W=8, scale=0.0625,
+             out=0x50000, out_stride_t=16 * 256, out_stride_h=256, nsplit=1, workspace=None,
+             workspace_bytes=0, err_word=None, stream=None)
+    a.update(over)
+    return qsa.qsa_sparse_prefill(**a)
+
+
+INVALID = [
+    (dict(q=None), qsa.QSA_ERR_INVALID_ARG),
+    (dict(k_cache=None), qsa.QSA_ERR_INVALID_ARG),
+    (dict(v_cache=None), qsa.QSA_ERR_INVALID_ARG),
+    (dict(out=None), qsa.QSA_ERR_INVALID_ARG),
+    (dict(slot_idx=None), qsa.QSA_ERR_INVALID_ARG),
+    (dict(q=0x10008), qsa.QSA_ERR_INVALID_ARG),          # misaligned base
+    (dict(out=0x50002), qsa.QSA_ERR_INVALID_ARG),
+    (dict(slot_idx=0x40002), qsa.QSA_ERR_INVALID_ARG),
+    (dict(width=0x60001), qsa.QSA_ERR_INVALID_ARG),
+    (dict(q_stride_h=260), qsa.QSA_ERR_INVALID_ARG),      # stride not a multiple of 8
+    (dict(k_stride_s=-512), qsa.QSA_ERR_INVALID_ARG),
+    (dict(out_stride_t=12), qsa.QSA_ERR_INVALID_ARG),
+    (dict(idx_stride_t=-1), qsa.QSA_ERR_INVALID_ARG),
+    (dict(Hkv=3), qsa.QSA_ERR_INVALID_ARG),
+    (dict(D=128), qsa.QSA_ERR_UNSUPPORTED),
+    (dict(Hq=34), qsa.QSA_ERR_UNSUPPORTED),               # G = 17
+    (dict(S=-1), qsa.QSA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), qsa.QSA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), qsa.QSA_ERR_INVALID_ARG),
+    (dict(nsplit=-2), qsa.QSA_ERR_INVALID_ARG),
+    (dict(nsplit=2, W=8, workspace=None), qsa.QSA_ERR_WORKSPACE),
+    (dict(nsplit=2, W=8, workspace=0x70000, workspace_bytes=16), qsa.QSA_ERR_WORKSPACE),
+]
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="fake-pointer validation runs only where no GPU can be reached")
+@pytest.mark.parametrize("over,status", INVALID, ids=[str(o) for o, _ in INVALID])
+def test_invalid_arguments_rejected_before_launch(lib, over, status):
+    assert _call(**over) == status
+    assert qsa.qsa_last_error_detail() != ""
+
+
+def test_empty_batch_is_a_noop(lib):
+    assert _call(Tq=0, q=None, k_cache=None, v_cache=None, out=None, slot_idx=None) == qsa.QSA_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_no_device_reports_cuda_error(lib):
+    # valid arguments, automatic split: the device query fails without a GPU
+    assert _call(nsplit=0) == qsa.QSA_ERR_CUDA
+
+
+def test_wrapper_refuses_cpu_tensors():
+    q = torch.zeros(2, 16, 256, dtype=torch.bfloat16)
+    k = torch.zeros(4, 2, 256, dtype=torch.bfloat16)
+    idx = torch.zeros(2, 3, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        qsa.sparse_prefill(q, k, k, idx)

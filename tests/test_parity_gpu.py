@@ -1,0 +1,321 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Gates (article "Qwen4-Exp QSA comes to Huawei's Ascend: inside SGLang's opt-in CANN
+prefill PR", section "Nine tests that passed, ..."): atol 0.025, rtol 0.025, rel-L2
+below 0.008, empty rows exactly zero, all outputs finite.  Small configurations are
+compared in full; the large ones are launched at full size in the configuration the
+benchmark times and compared on sampled rows (the article's long-prefill check used 8
+sampled rows; these tests use more).
+"""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import top_sparse_attention_index_b200 as qsa
+from helpers import check_gates, load_golden, valid_counts
+from top_sparse_attention_index_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+D = 256
+
+
+def dev(w: wl.Workload, device):
+    """Device copies that keep the layout (the width sweep's Q stays a strided view)."""
+    if w.q.is_contiguous():
+        q = w.q.to(device)
+    else:
+        base = w.q.as_strided((w.Tq, w.q.stride(0) // (w.Hq * D), w.Hq, D),
+                              (w.q.stride(0), w.Hq * D, D, 1))
+        q = base.to(device)[:, 0]
+        assert q.stride() == w.q.stride()
+    return dict(q=q, k_cache=w.k_cache.to(device), v_cache=w.v_cache.to(device),
+                slot_idx=w.slot_idx.to(device),
+                width=None if w.width is None else w.width.to(device))
+
+
+def run(d, scale, nsplit=0, **kw):
+    out = qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"], d["width"],
+                             scale=scale, nsplit=nsplit, **kw)
+    torch.cuda.synchronize()
+    return out.cpu()
+
+
+def empty_rows(w, rows=None):
+    cnt = valid_counts(w.slot_idx, w.width, w.S)
+    rows = range(w.Tq) if rows is None else rows
+    return [i for i, t in enumerate(rows) if int(cnt[t]) == 0]
+
+
+def compare_rows(w, got, oracle_lib, scale, rows, label):
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=rows)
+    return check_gates(got[rows].float(), torch.from_numpy(ref), empty_rows(w, rows), label)
+
+
+# ---- golden closed forms ------------------------------------------------------------
+
+def test_golden_closed_forms(cuda_device):
+    for c in load_golden():
+        d = dict(q=c["q"].to(cuda_device), k_cache=c["k"].to(cuda_device),
+                 v_cache=c["v"].to(cuda_device), slot_idx=c["slot_idx"].to(cuda_device),
+                 width=None if c["width"] is None else c["width"].to(cuda_device))
+        got = run(d, c["scale"])
+        empty = (c["expected"].abs().sum(dim=(1, 2)) == 0).nonzero().flatten().tolist()
+        check_gates(got.float(), c["expected"], empty, c["name"])
+
+
+# ---- the five configurations --------------------------------------------------------
+
+@pytest.mark.parametrize("nsplit", [0, 1, 2, 4])
+def test_tiny(cuda_device, oracle_lib, nsplit):
+    w = wl.tiny()
+    got = run(dev(w, cuda_device), 1.0 / 16.0, nsplit)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), w.notes["masked_rows"], "tiny")
+
+
+@pytest.fixture(scope="module")
+def width_sweep():
+    return wl.width_sweep()
+
+
+@pytest.mark.parametrize("scale", [1.0 / 16.0, 0.05])
+@pytest.mark.parametrize("nsplit", [0, 1, 3])
+def test_width_sweep(cuda_device, oracle_lib, width_sweep, scale, nsplit):
+    w = width_sweep
+    d = dev(w, cuda_device)
+    assert not d["q"].is_contiguous()
+    got = run(d, scale, nsplit)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale)
+    check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"width_sweep s={scale}")
+    # per-width gates as well (the article lists widths 1/63/64/65/2051 separately)
+    for k, wd in enumerate(wl.WIDTH_CYCLE):
+        rows = list(range(k, w.Tq, len(wl.WIDTH_CYCLE)))
+        check_gates(got[rows].float(), torch.from_numpy(ref[rows]), empty_rows(w, rows),
+                    f"width {wd}")
+
+
+def _causal_rows(Tq):
+    L = 8192
+    rows = set(range(0, 8)) | {L - 1, L, L + 1, L + 4095, L + 4096, Tq - 1}
+    rows |= {127, 128, 129, 2050, 2051, 2052}
+    rows |= {L + p for p in (127, 128, 2050, 2051, 5000)}
+    g = torch.Generator().manual_seed(5)
+    rows |= set(torch.randint(0, Tq, (96,), generator=g).tolist())
+    return sorted(r for r in rows if r < Tq)
+
+
+def test_causal_two_request(cuda_device, oracle_lib):
+    w = wl.causal_two_request()
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    assert torch.isfinite(got.float()).all()
+    rows = _causal_rows(w.Tq)
+    # the sampled rows cover every compression-ratio-4 tail remainder of the width
+    assert {int(w.width[r]) % 4 for r in rows} == {0, 1, 2, 3}
+    compare_rows(w, got, oracle_lib, 1.0 / 16.0, rows, "causal")
+
+
+def test_long_prefill_headline(cuda_device, oracle_lib):
+    """7,810 queries x 2,051 slots over 65,536 slots, launched as the benchmark does
+    (automatic plan); 8 evenly spaced rows as in the article plus 248 random rows."""
+    w = wl.long_prefill()
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    assert torch.isfinite(got.float()).all()
+    eight = [int(i * (w.Tq - 1) / 7) for i in range(8)]
+    compare_rows(w, got, oracle_lib, 1.0 / 16.0, eight, "long prefill, 8 rows")
+    g = torch.Generator().manual_seed(8)
+    rows = sorted(set(torch.randint(0, w.Tq, (248,), generator=g).tolist()) | set(eight))
+    compare_rows(w, got, oracle_lib, 1.0 / 16.0, rows, "long prefill, sampled")
+
+
+@pytest.mark.parametrize("Hq", [6, 3])
+@pytest.mark.parametrize("clustered", [False, True])
+def test_max_extent(cuda_device, oracle_lib, Hq, clustered):
+    w = wl.max_extent(Hq=Hq, clustered=clustered)
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    assert torch.isfinite(got.float()).all()
+    g = torch.Generator().manual_seed(9)
+    rows = sorted(set(torch.randint(0, w.Tq, (64,), generator=g).tolist()) | {0, w.Tq - 1})
+    compare_rows(w, got, oracle_lib, 1.0 / 16.0, rows, w.name)
+
+
+# ---- head shapes, row counts, split plans ---------------------------------------------
+
+def _random_case(seed, Tq, Hq, Hkv, S, W, minus1=0.0, widths=False):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(Tq, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    idx = wl.uniform_distinct(g, Tq, S, W)
+    if minus1:
+        idx[torch.rand(Tq, W, generator=g) < minus1] = -1
+    width = torch.randint(0, W + 1, (Tq,), generator=g, dtype=torch.int32) if widths else None
+    return wl.Workload(f"rand_{Hq}_{Hkv}_{Tq}", q, k, v, idx, width)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (24, 2), (12, 1), (6, 1), (3, 1), (16, 1), (5, 1), (2, 2)])
+@pytest.mark.parametrize("Tq", [1, 257])
+def test_head_shapes(cuda_device, oracle_lib, Hq, Hkv, Tq):
+    w = _random_case(1000 + Hq * 10 + Hkv + Tq, Tq, Hq, Hkv, 8192, 2051, minus1=0.05, widths=True)
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"heads ({Hq},{Hkv}) Tq={Tq}")
+
+
+@pytest.mark.parametrize("nsplit", [1, 2, 7, 16, 2051])
+def test_forced_splits_decode_shape(cuda_device, oracle_lib, nsplit):
+    """Few query rows with a wide selection: all the parallelism comes from splitting W,
+    down to one position per split."""
+    w = _random_case(77, 3, 16, 2, 65536, 2051, minus1=0.3)
+    got = run(dev(w, cuda_device), 1.0 / 16.0, nsplit)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"nsplit={nsplit}")
+
+
+def test_rows_wider_than_one_split(cuda_device, oracle_lib):
+    """W = 6,000 > 2,560 positions per split forces at least three splits."""
+    w = _random_case(78, 300, 16, 2, 20000, 6000, minus1=0.1, widths=True)
+    n, _ = qsa.qsa_sparse_prefill_plan(w.Tq, 16, 2, D, w.W, 148)
+    assert n >= 3
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    rows = list(range(0, w.Tq, 5))
+    compare_rows(w, got, oracle_lib, 1.0 / 16.0, rows, "W=6000")
+
+
+# ---- edge cases -----------------------------------------------------------------------
+
+def test_empty_rows_are_exact_zero(cuda_device):
+    w = _random_case(80, 40, 16, 2, 1000, 100)
+    w.slot_idx[::3] = -1                       # fully masked rows
+    w.width = torch.full((40,), 100, dtype=torch.int32)
+    w.width[1::3] = 0                          # zero selection width
+    for nsplit in (1, 4):
+        got = run(dev(w, cuda_device), 1.0 / 16.0, nsplit)
+        for t in list(range(0, 40, 3)) + list(range(1, 40, 3)):
+            assert (got[t].view(torch.int16) == 0).all(), t   # +0.0 bit patterns
+        assert (got[2::3].float().abs().sum(dim=(1, 2)) > 0).all()
+
+
+def test_zero_width_axis_and_empty_batch(cuda_device):
+    q = torch.randn(5, 16, D, device=cuda_device).to(torch.bfloat16)
+    kv = torch.randn(10, 2, D, device=cuda_device).to(torch.bfloat16)
+    idx = torch.empty(5, 0, dtype=torch.int32, device=cuda_device)
+    out = torch.full((5, 16, D), 7.0, dtype=torch.bfloat16, device=cuda_device)
+    qsa.sparse_prefill(q, kv, kv, idx, out=out)
+    torch.cuda.synchronize()
+    assert (out.view(torch.int16) == 0).all()
+    out0 = qsa.sparse_prefill(q[:0], kv, kv, idx[:0])
+    assert out0.shape == (0, 16, D)
+
+
+def test_width_one_returns_v_exactly(cuda_device):
+    w = _random_case(81, 64, 24, 2, 4096, 50)
+    w.width = torch.ones(64, dtype=torch.int32)
+    got = run(dev(w, cuda_device), 0.37)
+    for t in range(64):
+        s = int(w.slot_idx[t, 0])
+        for h in range(24):
+            assert torch.equal(got[t, h], w.v_cache[s, h // 12]), (t, h)
+
+
+def test_zero_query_rows_give_mean_of_v(cuda_device, oracle_lib):
+    """The 'zero rows' reading of an all-zero Q row: uniform weights, mean of V."""
+    w = _random_case(82, 32, 16, 2, 3000, 300, minus1=0.2)
+    w.q[::2] = 0
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), "zero q rows")
+    for t in range(0, 32, 2):
+        sel = [int(s) for s in w.slot_idx[t] if s >= 0]
+        mean = w.v_cache[sel].double().mean(dim=0)          # [Hkv, D]
+        assert torch.allclose(got[t].double(), mean.repeat_interleave(8, dim=0), atol=0.01)
+
+
+def test_invalid_slots_and_widths_set_error_bits(cuda_device, oracle_lib):
+    w = _random_case(83, 16, 16, 2, 500, 40, widths=True)
+    bad = w.slot_idx.clone()
+    bad[3, 0] = 500      # == S
+    bad[5, 2] = -9
+    wd = w.width.clone()
+    wd[7] = 41           # > W
+    wd[8] = -4
+    d = dev(w, cuda_device)
+    d["slot_idx"] = bad.to(cuda_device)
+    d["width"] = wd.to(cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    got = run(d, 1.0 / 16.0, err_word=err)
+    bits = int(err.item())
+    assert bits & qsa.QSA_ERRBIT_SLOT_RANGE and bits & qsa.QSA_ERRBIT_WIDTH_RANGE
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, bad, wd, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), None, "invalid slots")
+    clean = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    run(dev(w, cuda_device), 1.0 / 16.0, err_word=clean)
+    assert int(clean.item()) == 0
+
+
+def test_strided_kv_and_out_views(cuda_device, oracle_lib):
+    """K and V as views into one [S, 2, Hkv, D] buffer; out as a view of a wider
+    buffer: only the strides change."""
+    w = _random_case(84, 100, 16, 2, 2048, 300, minus1=0.1)
+    kv = torch.stack([w.k_cache, w.v_cache], dim=1).to(cuda_device)   # [S, 2, Hkv, D]
+    big = torch.zeros(100, 16, 2 * D, dtype=torch.bfloat16, device=cuda_device)
+    out = big[:, :, D:]
+    assert not out.is_contiguous()
+    qsa.sparse_prefill(w.q.to(cuda_device), kv[:, 0], kv[:, 1], w.slot_idx.to(cuda_device),
+                       scale=1.0 / 16.0, out=out)
+    torch.cuda.synchronize()
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
+    check_gates(out.cpu().float(), torch.from_numpy(ref), empty_rows(w), "strided views")
+    assert (big[:, :, :D] == 0).all()
+
+
+def test_deterministic_and_inputs_untouched(cuda_device):
+    """Cache-content reuse: the same call twice is bitwise identical; inputs unchanged."""
+    w = _random_case(85, 500, 16, 2, 16384, 2051, minus1=0.05)
+    d = dev(w, cuda_device)
+    before = [t.clone() for t in (d["q"], d["k_cache"], d["v_cache"], d["slot_idx"])]
+    a = run(d, 1.0 / 16.0)
+    b = run(d, 1.0 / 16.0)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    for x, y in zip(before, (d["q"], d["k_cache"], d["v_cache"], d["slot_idx"])):
+        assert torch.equal(x, y)
+
+
+def test_duplicate_slots_count_per_occurrence(cuda_device, oracle_lib):
+    w = _random_case(86, 20, 12, 1, 64, 48)
+    w.slot_idx[:, 24:] = w.slot_idx[:, :24]
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), None, "duplicates")
+
+
+def test_side_stream(cuda_device, oracle_lib):
+    w = _random_case(87, 64, 16, 2, 4096, 700)
+    d = dev(w, cuda_device)
+    s = torch.cuda.Stream(cuda_device)
+    with torch.cuda.stream(s):
+        out = qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"])
+    s.synchronize()
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
+    check_gates(out.cpu().float(), torch.from_numpy(ref), None, "side stream")
+
+
+def test_invalid_arguments_with_device_tensors(cuda_device):
+    q = torch.randn(4, 16, D, device=cuda_device).to(torch.bfloat16)
+    kv = torch.randn(10, 2, D, device=cuda_device).to(torch.bfloat16)
+    idx = torch.zeros(4, 3, dtype=torch.int32, device=cuda_device)
+    out = torch.full((4, 16, D), 3.0, dtype=torch.bfloat16, device=cuda_device)
+    # a q view whose base is not 16-byte aligned
+    qq = torch.randn(4 * 16 * D + 1, device=cuda_device).to(torch.bfloat16)[1:].view(4, 16, D)
+    with pytest.raises(qsa.QSAError) as ei:
+        qsa.sparse_prefill(qq, kv, kv, idx, out=out)
+    assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+    with pytest.raises(qsa.QSAError) as ei:
+        qsa.sparse_prefill(q[:, :15], kv, kv, idx[:, :], out=out[:, :15], scale=float("nan"))
+    assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+    with pytest.raises(qsa.QSAError) as ei:
+        qsa.sparse_prefill(q[:, :15], kv, kv, idx, out=out[:, :15])   # 15 % 2 != 0
+    assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert (out == 3.0).all()   # nothing was launched

@@ -1,0 +1,30 @@
+"""B200-native (sm_100a) Top-K-selected sparse attention for QSA prefill.
+
+The computation lives in libqsa.so (hand-written CUDA behind the C ABI in
+include/qsa.h); this package is its thin Python binding plus seeded workload
+generators.  Importing the package does not load the library; the first call does,
+and raises if the library is missing (there is no CPU fallback).
+"""
+from ._binding import (  # noqa: F401
+    QSA_ERR_CUDA,
+    QSA_ERR_INVALID_ARG,
+    QSA_ERR_UNSUPPORTED,
+    QSA_ERR_WORKSPACE,
+    QSA_ERRBIT_SLOT_RANGE,
+    QSA_ERRBIT_WIDTH_RANGE,
+    QSA_MAX_SLOTS_PER_SPLIT,
+    QSA_OK,
+    QSAError,
+    load_library,
+    qsa_abi_version,
+    qsa_last_error_detail,
+    qsa_sparse_prefill,
+    qsa_sparse_prefill_plan,
+    qsa_status_string,
+    sparse_prefill,
+)
+
+__all__ = [
+    "sparse_prefill", "qsa_sparse_prefill", "qsa_sparse_prefill_plan", "qsa_status_string",
+    "qsa_last_error_detail", "qsa_abi_version", "load_library", "QSAError",
+]

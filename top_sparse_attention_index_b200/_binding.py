@@ -1,0 +1,164 @@
+"""ctypes binding of libqsa.so: argument marshalling only.
+
+Every step of the computation runs in the CUDA kernels behind the C ABI declared in
+include/qsa.h; this module converts torch tensors into pointers, strides and the
+current CUDA stream, and turns status codes into exceptions.  There is no fallback:
+if the library is missing or a GPU is absent, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+LIBRARY = Path(__file__).resolve().parent / "libqsa.so"
+
+QSA_OK = 0
+QSA_ERR_INVALID_ARG = 1
+QSA_ERR_UNSUPPORTED = 2
+QSA_ERR_WORKSPACE = 3
+QSA_ERR_CUDA = 4
+QSA_ERRBIT_SLOT_RANGE = 0x1
+QSA_ERRBIT_WIDTH_RANGE = 0x2
+QSA_MAX_SLOTS_PER_SPLIT = 2560
+
+# Every symbol include/qsa.h declares, with its ctypes signature (restype, argtypes).
+_p, _i32, _i64, _sz, _f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+SIGNATURES = {
+    "qsa_abi_version": (_i32, []),
+    "qsa_sparse_prefill_plan": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]),
+    "qsa_sparse_prefill": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64, _p,
+                                  _i32, _i32, _i32, _i32, _i64, _i32, _f, _p, _i64, _i64, _i32,
+                                  _p, _sz, _p, _p]),
+    "qsa_status_string": (ctypes.c_char_p, [_i32]),
+    "qsa_last_error_detail": (ctypes.c_char_p, []),
+}
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{qsa_status_string(status)}: {detail}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library(path: Path | str | None = None):
+    """Load libqsa.so (built in-tree by build_lib.py); raises if it is missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    path = Path(path) if path is not None else LIBRARY
+    if not path.exists():
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m top_sparse_attention_index_b200.build_lib`")
+    lib = ctypes.CDLL(str(path))
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIBRARY:
+        _lib = lib
+    return lib
+
+
+# ---- names of the C ABI -------------------------------------------------------------
+
+def qsa_abi_version() -> int:
+    return int(load_library().qsa_abi_version())
+
+
+def qsa_status_string(status: int) -> str:
+    return load_library().qsa_status_string(int(status)).decode()
+
+
+def qsa_last_error_detail() -> str:
+    return load_library().qsa_last_error_detail().decode()
+
+
+def qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms, nsplit_request=0):
+    """(nsplit, workspace_bytes) for this shape; raises QSAError for invalid shapes."""
+    ws = ctypes.c_size_t(0)
+    n = int(load_library().qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms, nsplit_request,
+                                                   ctypes.byref(ws)))
+    if n < 0:
+        raise QSAError(-n, qsa_last_error_detail())
+    return n, int(ws.value)
+
+
+def qsa_sparse_prefill(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,
+                       v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S,
+                       W, scale, out, out_stride_t, out_stride_h, nsplit, workspace,
+                       workspace_bytes, err_word, stream) -> int:
+    """Raw call with integer pointers; returns the status code unchanged."""
+    return int(load_library().qsa_sparse_prefill(
+        q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache, v_stride_s,
+        v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W, ctypes.c_float(scale),
+        out, out_stride_t, out_stride_h, nsplit, workspace, workspace_bytes, err_word, stream))
+
+
+# ---- torch-facing wrapper ------------------------------------------------------------
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_dev(name, t, dtype, device):
+    if t.device != device:
+        raise ValueError(f"{name} must live on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() > 0 and t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name} must be contiguous in its last dimension")
+
+
+def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=None, nsplit=0,
+                   err_word=None, stream=None):
+    """Selected-slot sparse attention on the GPU.
+
+    q [Tq, Hq, 256] bf16, k_cache / v_cache [S, Hkv, 256] bf16, slot_idx [Tq, W] int32
+    (-1 = masked), width [Tq] int32 or None; scale defaults to 1/sqrt(256) = 1/16.
+    Returns out [Tq, Hq, 256] bf16 (allocated unless given).  Work is enqueued on
+    ``stream`` (default: torch's current stream); nothing is synchronised.
+    """
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("sparse_prefill runs on CUDA tensors only")
+    Tq, Hq, D = q.shape
+    S, Hkv, Dk = k_cache.shape
+    if Dk != D or tuple(v_cache.shape) != (S, Hkv, D):
+        raise ValueError("k_cache and v_cache must both be [S, Hkv, D]")
+    if slot_idx.dim() != 2 or slot_idx.shape[0] != Tq:
+        raise ValueError("slot_idx must be [Tq, W]")
+    W = slot_idx.shape[1]
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
+                        ("v_cache", v_cache, torch.bfloat16), ("slot_idx", slot_idx, torch.int32)):
+        _check_dev(name, t, dt, device)
+    if width is not None:
+        _check_dev("width", width, torch.int32, device)
+        if tuple(width.shape) != (Tq,) or (Tq > 1 and width.stride(0) != 1):
+            raise ValueError("width must be a contiguous [Tq] int32 tensor")
+    if out is None:
+        out = torch.empty(Tq, Hq, D, dtype=torch.bfloat16, device=device)
+    else:
+        _check_dev("out", out, torch.bfloat16, device)
+        if tuple(out.shape) != (Tq, Hq, D):
+            raise ValueError("out must be [Tq, Hq, D]")
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    num_sms = torch.cuda.get_device_properties(device).multi_processor_count
+    ns, ws_bytes = qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms, nsplit)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device) if ws_bytes else None
+    with torch.cuda.device(device):
+        st = qsa_sparse_prefill(
+            _ptr(q), q.stride(0), q.stride(1), _ptr(k_cache), k_cache.stride(0), k_cache.stride(1),
+            _ptr(v_cache), v_cache.stride(0), v_cache.stride(1), _ptr(slot_idx) if W else None,
+            slot_idx.stride(0), _ptr(width), Tq, Hq, Hkv, D, S, W, float(scale), _ptr(out),
+            out.stride(0), out.stride(1), ns, _ptr(ws), ws_bytes, _ptr(err_word), stream.cuda_stream)
+    if st != QSA_OK:
+        raise QSAError(st, qsa_last_error_detail())
+    return out

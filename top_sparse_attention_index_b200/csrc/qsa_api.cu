@@ -1,0 +1,206 @@
+// qsa_api.cu -- the C ABI of libqsa.so: argument validation, the split planner and the
+// launch.  Declarations and the full contract are in include/qsa.h.
+//
+// The host side never synchronises and never allocates: every check below uses only
+// the scalar arguments and pointer values, so a call is a pure enqueue on `stream`
+// (unlike the Ascend adapter described in "What the pull request actually adds",
+// whose extent check copies two scalars to the host).
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+
+#include "qsa.h"
+#include "qsa_internal.h"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+qsa_status_t fail(qsa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+struct Plan {
+  int32_t nsplit;
+  int32_t split_len;
+  size_t workspace;
+};
+
+// Shape validation shared by the planner and the launch; returns QSA_OK or an error.
+qsa_status_t check_shape(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W) {
+  if (Tq < 0 || W < 0) return fail(QSA_ERR_INVALID_ARG, "negative size: Tq=%d W=%d", Tq, W);
+  if (Hq <= 0 || Hkv <= 0 || D <= 0)
+    return fail(QSA_ERR_INVALID_ARG, "non-positive size: Hq=%d Hkv=%d D=%d", Hq, Hkv, D);
+  if (Hq % Hkv != 0) return fail(QSA_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  if (D != qsa::kHeadDim) return fail(QSA_ERR_UNSUPPORTED, "head dimension %d (only 256)", D);
+  const int32_t G = Hq / Hkv;
+  if (G > qsa::kMaxGroup) return fail(QSA_ERR_UNSUPPORTED, "group size G=%d (1..16)", G);
+  return QSA_OK;
+}
+
+Plan make_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W, int32_t num_sms, int32_t request) {
+  const int32_t G = Hq / Hkv;
+  const int32_t min_split = W > 0 ? (W + qsa::kMaxSlotsPerSplit - 1) / qsa::kMaxSlotsPerSplit : 1;
+  const int32_t max_split = W > 0 ? W : 1;
+  int32_t n;
+  if (request > 0) {
+    n = request < min_split ? min_split : (request > max_split ? max_split : request);
+  } else {
+    // Enough CTAs for about two waves; never splits narrower than kMinSlotsPerSplit.
+    const qsa::KernelShape ks = qsa::kernel_shape(G);
+    const int64_t wave = int64_t(num_sms > 0 ? num_sms : 1) * ks.ctas_per_sm;
+    const int64_t units = int64_t(Tq) * Hkv;
+    n = min_split;
+    if (units > 0 && units < 2 * wave) {
+      const int64_t want = (2 * wave + units - 1) / units;
+      const int64_t cap = W >= qsa::kMinSlotsPerSplit ? W / qsa::kMinSlotsPerSplit : 1;
+      const int64_t pick = want < cap ? want : cap;
+      if (pick > n) n = int32_t(pick);
+    }
+  }
+  int32_t split_len = W > 0 ? (W + n - 1) / n : 0;
+  if (W > 0) n = (W + split_len - 1) / split_len;  // no split lies wholly past W
+  return {n, split_len, qsa::workspace_bytes_for(Tq, Hq, n)};
+}
+
+int32_t device_sm_count(int dev) {
+  static std::atomic<int32_t> cache[64];
+  if (dev >= 0 && dev < 64) {
+    const int32_t c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 64) cache[dev].store(sms, std::memory_order_relaxed);
+  return sms;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool stride_ok(int64_t s) { return s >= 0 && (s % 8) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t qsa_abi_version(void) { return 1; }
+
+const char* qsa_status_string(qsa_status_t status) {
+  switch (status) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
+    case QSA_ERR_WORKSPACE: return "QSA_ERR_WORKSPACE";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+  }
+  return "QSA_ERR_UNKNOWN";
+}
+
+const char* qsa_last_error_detail(void) { return g_detail; }
+
+int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W,
+                                int32_t num_sms, int32_t nsplit_request,
+                                size_t* workspace_bytes) {
+  const qsa_status_t st = check_shape(Tq, Hq, Hkv, D, W);
+  if (st != QSA_OK) return -int32_t(st);
+  if (nsplit_request < 0) return -int32_t(fail(QSA_ERR_INVALID_ARG, "negative nsplit request"));
+  const Plan pl = make_plan(Tq, Hq, Hkv, W, num_sms, nsplit_request);
+  if (workspace_bytes != nullptr) *workspace_bytes = pl.workspace;
+  return pl.nsplit;
+}
+
+qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                const int32_t* slot_idx, int64_t idx_stride_t,
+                                const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                int32_t D, int64_t S, int32_t W, float scale, void* out,
+                                int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
+                                void* workspace, size_t workspace_bytes, uint32_t* err_word,
+                                void* stream) {
+  g_detail[0] = '\0';
+  qsa_status_t st = check_shape(Tq, Hq, Hkv, D, W);
+  if (st != QSA_OK) return st;
+  if (S < 0) return fail(QSA_ERR_INVALID_ARG, "negative S");
+  if (nsplit < 0) return fail(QSA_ERR_INVALID_ARG, "negative nsplit");
+  if (!std::isfinite(scale)) return fail(QSA_ERR_INVALID_ARG, "scale is not finite");
+  if (Tq == 0) return QSA_OK;
+
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr)
+    return fail(QSA_ERR_INVALID_ARG, "NULL q, k_cache, v_cache or out");
+  if (W > 0 && slot_idx == nullptr) return fail(QSA_ERR_INVALID_ARG, "NULL slot_idx with W > 0");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return fail(QSA_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
+  if ((slot_idx != nullptr && !aligned4(slot_idx)) || (width != nullptr && !aligned4(width)) ||
+      (err_word != nullptr && !aligned4(err_word)))
+    return fail(QSA_ERR_INVALID_ARG, "slot_idx, width and err_word must be 4-byte aligned");
+  if (!stride_ok(q_stride_t) || !stride_ok(q_stride_h) || !stride_ok(k_stride_s) ||
+      !stride_ok(k_stride_h) || !stride_ok(v_stride_s) || !stride_ok(v_stride_h) ||
+      !stride_ok(out_stride_t) || !stride_ok(out_stride_h))
+    return fail(QSA_ERR_INVALID_ARG, "tensor strides must be non-negative multiples of 8 elements");
+  if (idx_stride_t < 0) return fail(QSA_ERR_INVALID_ARG, "negative idx_stride_t");
+
+  int32_t num_sms = 0;
+  if (nsplit == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    num_sms = device_sm_count(dev);
+    if (num_sms <= 0) return fail(QSA_ERR_CUDA, "cannot query the multiprocessor count");
+  }
+  const Plan pl = make_plan(Tq, Hq, Hkv, W, num_sms, nsplit);
+  if (int64_t(Tq) * Hkv * pl.nsplit > int64_t(INT32_MAX))
+    return fail(QSA_ERR_INVALID_ARG, "too many work units for one launch");
+  if (pl.workspace > 0) {
+    if (workspace == nullptr || workspace_bytes < pl.workspace)
+      return fail(QSA_ERR_WORKSPACE, "workspace of %zu bytes needed for nsplit=%d, got %zu",
+                  pl.workspace, pl.nsplit, workspace == nullptr ? size_t(0) : workspace_bytes);
+    if (!aligned16(workspace)) return fail(QSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  }
+
+  qsa::FwdParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k_cache = static_cast<const uint16_t*>(k_cache);
+  p.v_cache = static_cast<const uint16_t*>(v_cache);
+  p.slot_idx = slot_idx;
+  p.width = width;
+  p.out = static_cast<uint16_t*>(out);
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = pl.workspace > 0
+                 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                            qsa::workspace_lse_offset(Tq, Hq, pl.nsplit))
+                 : nullptr;
+  p.err_word = err_word;
+  p.q_stride_t = q_stride_t;
+  p.q_stride_h = q_stride_h;
+  p.k_stride_s = k_stride_s;
+  p.k_stride_h = k_stride_h;
+  p.v_stride_s = v_stride_s;
+  p.v_stride_h = v_stride_h;
+  p.idx_stride_t = idx_stride_t;
+  p.out_stride_t = out_stride_t;
+  p.out_stride_h = out_stride_h;
+  p.S = S;
+  p.Tq = Tq;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.W = W;
+  p.nsplit = pl.nsplit;
+  p.split_len = pl.split_len;
+  p.scale_log2 = scale * 1.4426950408889634f;  // log2(e): the kernels use 2^x
+
+  const cudaError_t e = qsa::launch_sparse_prefill(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return QSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,440 @@
+// qsa_attn.cu -- sm_100a kernels for selected-slot sparse attention (QSA prefill).
+//
+// Operation (article "Qwen4-Exp QSA comes to Huawei's Ascend: inside SGLang's opt-in
+// CANN prefill PR", section "What the pull request actually adds"): for every query row
+// t and KV head j, gather the row's selected physical slots of K and V, form
+// scale * Q K^T for the whole GQA group of G = Hq / Hkv query heads, take the softmax
+// over the selected slots only and return P V; a row without a valid slot returns 0.
+//
+// K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit:
+//   1. stage the split's slot indices in shared memory and compact away -1 (and
+//      out-of-range) entries with a block scan, so masked slots cost no bandwidth;
+//   2. gather K and V rows of the compacted slots with 16-byte cp.async into a
+//      STAGES-deep shared-memory ring (row = 512 contiguous bytes; the 16-byte chunks
+//      of a row are XOR-swizzled by the row index so ldmatrix reads are conflict-free);
+//   3. per warp and 16-slot sub-tile: S^T = K Q^T with the slots as the MMA M dimension
+//      and the (up to 8) heads of one n8 tile as N, so the group shares every gathered
+//      row and G = 3/6/8/12/16 needs no padding of the head ratio in memory;
+//      online softmax in fp32 registers (base 2, warp shuffles over the slot axis);
+//      P rounded to bf16 and transposed in registers (movmatrix) into the B operand of
+//      O^T += V^T P^T with D = 256 as M;
+//   4. merge the per-warp (m, l, O) states through shared memory and write bf16 out
+//      (exact zeros for empty rows), or fp32 partials + base-2 LSE when split.
+// K2 qsa_lse_combine_kernel -- one warp per (t, h): log-sum-exp weighted sum of the
+//   split partials; empty splits carry LSE = -inf and weight 0; all empty -> exact 0.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "qsa_internal.h"
+#include "qsa_ptx.cuh"
+
+namespace qsa {
+namespace {
+
+constexpr int kRowBytes = kHeadDim * 2;     // one (slot, head) row: 512 bytes
+constexpr int kChunks = kRowBytes / 16;     // 32 16-byte chunks per row
+constexpr int kMergeStride = kHeadDim + 4;  // padded fp32 row of the epilogue merge
+constexpr float kNegInf = -__builtin_huge_valf();
+
+template <int NTILE, int SL, int STAGES>
+struct Cfg {
+  static constexpr int kWarps = NTILE * SL;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kRows = 16 * SL;                      // slots per stage
+  static constexpr int kStageBytes = kRows * kRowBytes * 2;  // K rows then V rows
+  static constexpr int kRingBytes = STAGES * kStageBytes;
+  static constexpr int kQBytes = NTILE * 8 * kRowBytes;
+  static constexpr int kIdxBytes = kMaxSlotsPerSplit * 4;
+  static constexpr int kScanBytes = 32 * 4;
+  static constexpr int kMergeBytes = kWarps * (8 * kMergeStride + 16) * 4;
+  static constexpr size_t kSmem = size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes;
+  static_assert(kMergeBytes <= kRingBytes, "merge buffer reuses the ring");
+  static_assert(kIdxBytes <= kRingBytes, "raw index staging reuses the ring");
+  static_assert(kRows % kWarps == 0, "each warp loads whole rows");
+};
+
+template <int NTILE, int SL, int STAGES>
+__global__ void __launch_bounds__(32 * NTILE * SL, 1)
+    qsa_sparse_attn_fwd_kernel(const FwdParams p) {
+  using C = Cfg<NTILE, SL, STAGES>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* ring = smem;
+  uint8_t* sQ = smem + C::kRingBytes;
+  int32_t* sIdx = reinterpret_cast<int32_t*>(sQ + C::kQBytes);
+  int32_t* sScan = sIdx + kMaxSlotsPerSplit;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int wslot = warp % SL;  // which 16-slot sub-tile of a stage
+  const int wn = warp / SL;     // which n8 tile of the head group
+
+  // ---- work unit -------------------------------------------------------------------
+  int u = blockIdx.x;
+  const int split = u % p.nsplit;
+  u /= p.nsplit;
+  const int j = u % p.Hkv;
+  const int t = u / p.Hkv;
+
+  int width_t = p.W;
+  if (p.width != nullptr) {
+    int wv = p.width[t];
+    if (wv < 0 || wv > p.W) {
+      if (tid == 0 && p.err_word != nullptr) atomicOr(p.err_word, 2u);
+      wv = wv < 0 ? 0 : p.W;
+    }
+    width_t = wv;
+  }
+  const int w0 = split * p.split_len;
+  const int n_raw = max(min(w0 + p.split_len, width_t) - w0, 0);
+
+  // ---- 1. stage and compact the slot indices -----------------------------------------
+  int32_t* sRaw = reinterpret_cast<int32_t*>(ring);
+  {
+    const int32_t* idx_row = p.slot_idx + int64_t(t) * p.idx_stride_t + w0;
+    for (int i = tid; i < n_raw; i += C::kThreads) sRaw[i] = __ldg(idx_row + i);
+  }
+  __syncthreads();
+  const int per = (n_raw + C::kThreads - 1) / C::kThreads;
+  const int b_i = min(tid * per, n_raw);
+  const int e_i = min(b_i + per, n_raw);
+  int cnt = 0;
+  bool bad = false;
+  for (int i = b_i; i < e_i; ++i) {
+    const int v = sRaw[i];
+    const bool ok = v >= 0 && int64_t(v) < p.S;
+    bad |= (!ok && v != -1);
+    cnt += ok ? 1 : 0;
+  }
+  if (bad && p.err_word != nullptr) atomicOr(p.err_word, 1u);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sScan[warp] = incl;
+  __syncthreads();
+  int n_valid = 0, warp_off = 0;
+#pragma unroll
+  for (int w = 0; w < C::kWarps; ++w) {
+    const int s = sScan[w];
+    warp_off += (w < warp) ? s : 0;
+    n_valid += s;
+  }
+  {
+    int pos = warp_off + incl - cnt;
+    for (int i = b_i; i < e_i; ++i) {
+      const int v = sRaw[i];
+      if (v >= 0 && int64_t(v) < p.S) sIdx[pos++] = v;
+    }
+  }
+  __syncthreads();  // sIdx complete, the ring is free again
+
+  const int G = p.G;
+  const int64_t head0 = int64_t(j) * G;
+  if (n_valid == 0) {  // fully masked row, zero width or an empty split (block-uniform)
+    if (p.nsplit == 1) {
+      for (int i = tid; i < G * kChunks; i += C::kThreads) {
+        const int g = i / kChunks, c = i % kChunks;
+        uint16_t* dst = p.out + int64_t(t) * p.out_stride_t + (head0 + g) * p.out_stride_h + c * 8;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else {
+      for (int g = tid; g < G; g += C::kThreads)
+        p.ws_lse[(int64_t(split) * p.Tq + t) * p.Hq + head0 + g] = kNegInf;
+    }
+    return;
+  }
+
+  // ---- 2. Q tile (group 0) and the pipeline prologue ------------------------------------
+  const uint32_t ring_s = smem_addr(ring);
+  const uint32_t q_s = smem_addr(sQ);
+  for (int i = tid; i < NTILE * 8 * kChunks; i += C::kThreads) {
+    const int g = i / kChunks, c = i % kChunks;
+    const bool ok = g < G;
+    const uint16_t* src =
+        p.q + int64_t(t) * p.q_stride_t + (head0 + (ok ? g : 0)) * p.q_stride_h + c * 8;
+    cp_async_16(q_s + g * kRowBytes + ((c ^ (g & 7)) << 4), src, ok);
+  }
+  cp_async_commit();
+
+  const int n_stages = (n_valid + C::kRows - 1) / C::kRows;
+  const uint16_t* kbase = p.k_cache + int64_t(j) * p.k_stride_h;
+  const uint16_t* vbase = p.v_cache + int64_t(j) * p.v_stride_h;
+  const int ld_chunk = lane;  // each warp moves whole 512-byte rows, one chunk per lane
+
+  auto load_stage = [&](int s, int buf) {
+    const uint32_t kdst = ring_s + buf * C::kStageBytes;
+    const uint32_t vdst = kdst + C::kRows * kRowBytes;
+#pragma unroll
+    for (int i = 0; i < C::kRows / C::kWarps; ++i) {
+      const int r = warp + i * C::kWarps;
+      const int pos = s * C::kRows + r;
+      const bool ok = pos < n_valid;
+      const int64_t slot = ok ? sIdx[pos] : 0;
+      const uint32_t off = r * kRowBytes + ((ld_chunk ^ (r & 7)) << 4);
+      cp_async_16(kdst + off, kbase + slot * p.k_stride_s + ld_chunk * 8, ok);
+      cp_async_16(vdst + off, vbase + slot * p.v_stride_s + ld_chunk * 8, ok);
+    }
+  };
+
+#pragma unroll
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < n_stages) load_stage(s, s);
+    cp_async_commit();
+  }
+  cp_async_wait<STAGES - 1>();  // the Q group is the oldest
+  __syncthreads();
+
+  // B fragments of Q^T for this warp's n8 tile, all 16 k-steps of D = 256.
+  uint32_t qf[16][2];
+#pragma unroll
+  for (int kp = 0; kp < 8; ++kp) {
+    const int g = lane & 7;
+    const int c = 4 * kp + (lane >> 3);
+    uint32_t r[4];
+    ldmatrix_x4(r, q_s + (wn * 8 + g) * kRowBytes + ((c ^ g) << 4));
+    qf[2 * kp][0] = r[0];
+    qf[2 * kp][1] = r[1];
+    qf[2 * kp + 1][0] = r[2];
+    qf[2 * kp + 1][1] = r[3];
+  }
+
+  // ---- 3. main loop ------------------------------------------------------------------
+  float m0 = kNegInf, m1 = kNegInf;  // running max (base 2) of heads 2(l%4), 2(l%4)+1
+  float l0 = 0.f, l1 = 0.f;          // this lane's share of the running sums
+  float o[16][4];
+#pragma unroll
+  for (int mt = 0; mt < 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+  const int key = lane & 7;  // swizzle key of every row this lane addresses
+  const int krow = wslot * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int khi = lane >> 4;
+  const int vrow = wslot * 16 + (lane & 7) + ((lane >> 4) << 3);
+  const int vhi = (lane >> 3) & 1;
+  const float sl2 = p.scale_log2;
+
+  for (int s = 0; s < n_stages; ++s) {
+    cp_async_wait<STAGES - 2>();
+    __syncthreads();
+    {
+      const int sn = s + STAGES - 1;
+      if (sn < n_stages) load_stage(sn, sn % STAGES);
+      cp_async_commit();
+    }
+    const int buf = s % STAGES;
+    const int base = s * C::kRows + wslot * 16;
+    if (base >= n_valid) continue;  // warp-uniform: no valid slot in this sub-tile
+
+    // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8); two chains for ILP.
+    const uint32_t kt = ring_s + buf * C::kStageBytes + krow * kRowBytes;
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 16; ks += 2) {
+      uint32_t a[4];
+      ldmatrix_x4(a, kt + (((2 * ks + khi) ^ key) << 4));
+      mma_bf16_16816(sa, a, qf[ks][0], qf[ks][1]);
+      ldmatrix_x4(a, kt + (((2 * ks + 2 + khi) ^ key) << 4));
+      mma_bf16_16816(sb, a, qf[ks + 1][0], qf[ks + 1][1]);
+    }
+    float x0 = (sa[0] + sb[0]) * sl2, x1 = (sa[1] + sb[1]) * sl2;
+    float x2 = (sa[2] + sb[2]) * sl2, x3 = (sa[3] + sb[3]) * sl2;
+    const int r0 = base + (lane >> 2);
+    if (r0 >= n_valid) x0 = x1 = kNegInf;
+    if (r0 + 8 >= n_valid) x2 = x3 = kNegInf;
+
+    // online softmax over the slot axis (rows): lanes sharing l%4 hold one head pair
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: row `base` is valid
+    const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    const uint32_t p01 = pack_bf16x2(fast_exp2(x0 - mn0), fast_exp2(x1 - mn1));
+    const uint32_t p23 = pack_bf16x2(fast_exp2(x2 - mn0), fast_exp2(x3 - mn1));
+    // the denominators sum the same bf16-rounded weights that multiply V
+    l0 = l0 * al0 + (bf16lo_to_f32(p01) + bf16lo_to_f32(p23));
+    l1 = l1 * al1 + (bf16hi_to_f32(p01) + bf16hi_to_f32(p23));
+    if (!__all_sync(0xffffffffu, al0 == 1.f && al1 == 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < 16; ++mt) {
+        o[mt][0] *= al0;
+        o[mt][1] *= al1;
+        o[mt][2] *= al0;
+        o[mt][3] *= al1;
+      }
+    }
+
+    // O^T (256 x 8) += V^T (256 x 16) * P^T (16 x 8)
+    const uint32_t b0 = movmatrix_trans(p01);
+    const uint32_t b1 = movmatrix_trans(p23);
+    const uint32_t vt = ring_s + buf * C::kStageBytes + C::kRows * kRowBytes + vrow * kRowBytes;
+#pragma unroll
+    for (int mt = 0; mt < 16; ++mt) {
+      uint32_t a[4];
+      ldmatrix_x4_trans(a, vt + (((2 * mt + vhi) ^ key) << 4));
+      mma_bf16_16816(o[mt], a, b0, b1);
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();  // every warp is done with the ring: reuse it for the merge
+
+  // ---- 4. merge the warps of each n8 tile and write ------------------------------------
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  float* mbuf = reinterpret_cast<float*>(ring);
+  constexpr int kWarpFloats = 8 * kMergeStride + 16;
+  {
+    float* mine = mbuf + warp * kWarpFloats;
+    const int g0 = 2 * (lane & 3);
+    const int r8 = lane >> 2;
+#pragma unroll
+    for (int mt = 0; mt < 16; ++mt) {
+      const int d = 16 * mt + r8;
+      mine[g0 * kMergeStride + d] = o[mt][0];
+      mine[(g0 + 1) * kMergeStride + d] = o[mt][1];
+      mine[g0 * kMergeStride + d + 8] = o[mt][2];
+      mine[(g0 + 1) * kMergeStride + d + 8] = o[mt][3];
+    }
+    if (r8 == 0) {
+      mine[8 * kMergeStride + g0] = m0;
+      mine[8 * kMergeStride + g0 + 1] = m1;
+      mine[8 * kMergeStride + 8 + g0] = l0;
+      mine[8 * kMergeStride + 8 + g0 + 1] = l1;
+    }
+  }
+  __syncthreads();
+
+  for (int it = tid; it < NTILE * 8 * 32; it += C::kThreads) {
+    const int gg = it >> 5;  // head within the group (n-tile major)
+    const int dg = it & 31;  // 8-wide d group
+    if (gg >= G) continue;
+    const int nt = gg >> 3, g = gg & 7;
+    float mstar = kNegInf;
+#pragma unroll
+    for (int w = 0; w < SL; ++w)
+      mstar = fmaxf(mstar, mbuf[(nt * SL + w) * kWarpFloats + 8 * kMergeStride + g]);
+    float lsum = 0.f;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int w = 0; w < SL; ++w) {
+      const float* src = mbuf + (nt * SL + w) * kWarpFloats;
+      const float sc = fast_exp2(src[8 * kMergeStride + g] - mstar);  // -inf -> 0
+      lsum += sc * src[8 * kMergeStride + 8 + g];
+      const float4 a = *reinterpret_cast<const float4*>(src + g * kMergeStride + dg * 8);
+      const float4 b = *reinterpret_cast<const float4*>(src + g * kMergeStride + dg * 8 + 4);
+      acc[0] += sc * a.x; acc[1] += sc * a.y; acc[2] += sc * a.z; acc[3] += sc * a.w;
+      acc[4] += sc * b.x; acc[5] += sc * b.y; acc[6] += sc * b.z; acc[7] += sc * b.w;
+    }
+    const float inv = 1.f / lsum;
+    const int64_t h = head0 + gg;
+    if (p.nsplit == 1) {
+      uint4 v;
+      v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+      v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+      *reinterpret_cast<uint4*>(p.out + int64_t(t) * p.out_stride_t + h * p.out_stride_h + dg * 8) = v;
+    } else {
+      const int64_t row = (int64_t(split) * p.Tq + t) * p.Hq + h;
+      float4* dst = reinterpret_cast<float4*>(p.ws_o + row * kHeadDim + dg * 8);
+      dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+      if (dg == 0) p.ws_lse[row] = mstar + fast_log2(lsum);
+    }
+  }
+}
+
+// K2: out[t, h, :] = sum_s 2^(lse_s - lse*) O_s / sum_s 2^(lse_s - lse*), one warp per row.
+__global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p) {
+  const int64_t rows = int64_t(p.Tq) * p.Hq;
+  const int64_t row = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  float mstar = kNegInf;
+  for (int s = 0; s < p.nsplit; ++s) mstar = fmaxf(mstar, p.ws_lse[s * rows + row]);
+  const int64_t t = row / p.Hq, h = row % p.Hq;
+  uint4* dst = reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8);
+  if (mstar == kNegInf) {
+    *dst = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < p.nsplit; ++s) {
+    const float lse = p.ws_lse[s * rows + row];
+    if (lse == kNegInf) continue;  // empty split: its partial was never written
+    const float w = fast_exp2(lse - mstar);
+    wsum += w;
+    const float4* src = reinterpret_cast<const float4*>(p.ws_o + (s * rows + row) * kHeadDim + lane * 8);
+    const float4 a = src[0], b = src[1];
+    acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+    acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
+  }
+  const float inv = 1.f / wsum;
+  uint4 v;
+  v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *dst = v;
+}
+
+template <int NTILE, int SL, int STAGES>
+cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
+  using C = Cfg<NTILE, SL, STAGES>;
+  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, SL, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(int64_t(p.Tq) * p.Hkv * p.nsplit);
+  kern<<<grid, C::kThreads, C::kSmem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+// The two shapes: G <= 8 (one n8 tile, 4 slot lanes, 64-slot stages, 3 stages) and
+// 8 < G <= 16 (two n8 tiles, 2 slot lanes, 32-slot stages, 6 stages).
+using CfgSmall = Cfg<1, 4, 3>;
+using CfgLarge = Cfg<2, 2, 6>;
+
+}  // namespace
+
+KernelShape kernel_shape(int G) {
+  if (G <= 8) return {1, 4, CfgSmall::kThreads, CfgSmall::kRows, 3, CfgSmall::kSmem, 1};
+  return {2, 2, CfgLarge::kThreads, CfgLarge::kRows, 6, CfgLarge::kSmem, 1};
+}
+
+size_t workspace_lse_offset(int32_t Tq, int32_t Hq, int32_t nsplit) {
+  const size_t o_bytes = size_t(nsplit) * size_t(Tq) * size_t(Hq) * kHeadDim * sizeof(float);
+  return (o_bytes + 255) / 256 * 256;
+}
+
+size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
+  if (nsplit <= 1) return 0;
+  const size_t lse_bytes = size_t(nsplit) * size_t(Tq) * size_t(Hq) * sizeof(float);
+  return workspace_lse_offset(Tq, Hq, nsplit) + (lse_bytes + 255) / 256 * 256;
+}
+
+cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
+  cudaError_t e = (p.G <= 8) ? launch_fwd<1, 4, 3>(p, stream) : launch_fwd<2, 2, 6>(p, stream);
+  if (e != cudaSuccess || p.nsplit == 1) return e;
+  const int64_t rows = int64_t(p.Tq) * p.Hq;
+  const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
+  qsa_lse_combine_kernel<<<grid, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

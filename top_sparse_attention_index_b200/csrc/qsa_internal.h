@@ -1,0 +1,59 @@
+// qsa_internal.h -- launch-side interface between the C ABI (qsa_api.cu) and the
+// kernels (qsa_attn.cu).  Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace qsa {
+
+constexpr int kHeadDim = 256;           // D: the only head dimension implemented
+constexpr int kMaxGroup = 16;           // largest G = Hq / Hkv
+constexpr int kMaxSlotsPerSplit = 2560; // per-split index list staged in shared memory
+constexpr int kMinSlotsPerSplit = 128;  // the planner never makes splits narrower
+
+// Everything one launch of the fused kernel needs (passed by value).
+struct FwdParams {
+  const uint16_t* q;        // bf16 bits [Tq, Hq, D]
+  const uint16_t* k_cache;  // bf16 bits [S, Hkv, D]
+  const uint16_t* v_cache;
+  const int32_t* slot_idx;  // [Tq, W] row stride idx_stride_t
+  const int32_t* width;     // [Tq] or nullptr
+  uint16_t* out;            // bf16 bits [Tq, Hq, D]
+  float* ws_o;              // fp32 [nsplit, Tq, Hq, D] (nsplit > 1)
+  float* ws_lse;            // fp32 [nsplit, Tq, Hq] base-2 log-sum-exp (nsplit > 1)
+  uint32_t* err_word;       // optional
+  int64_t q_stride_t, q_stride_h;
+  int64_t k_stride_s, k_stride_h;
+  int64_t v_stride_s, v_stride_h;
+  int64_t idx_stride_t;
+  int64_t out_stride_t, out_stride_h;
+  int64_t S;
+  int32_t Tq, Hq, Hkv, G, W;
+  int32_t nsplit;
+  int32_t split_len;        // positions of the W axis per split
+  float scale_log2;         // scale * log2(e)
+};
+
+// Kernel configuration chosen for a group size G (shared by planner and launcher).
+struct KernelShape {
+  int ntile;        // n8 tiles covering G (1 or 2)
+  int slot_lanes;   // warps along the slot axis
+  int threads;
+  int stage_rows;   // selected slots per pipeline stage
+  int stages;
+  size_t smem_bytes;
+  int ctas_per_sm;  // expected residency (for the planner)
+};
+
+KernelShape kernel_shape(int G);
+
+// Enqueue the fused kernel (and the combine when nsplit > 1) on `stream`.
+cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream);
+
+size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit);
+size_t workspace_lse_offset(int32_t Tq, int32_t Hq, int32_t nsplit);
+
+}  // namespace qsa

@@ -42,13 +42,15 @@ L2_FLUSH_BYTES = 512 << 20
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="keep only the first ROWS query rows (small cases for ncu captures)")
     return ap.parse_args()
 
 
@@ -77,7 +79,7 @@ def measured_peaks():
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -91,7 +93,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -108,13 +110,22 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [l for l in out.splitlines() if l.strip()]
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and the throttle reasons seen between wall times t0 and t1."""
+        import datetime
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in getattr(self, "lines", []):
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
+            if t0 is not None:
+                try:
+                    ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    ts = None
+                if ts is not None and not (t0 - 0.06 <= ts <= t1 + 0.06):
+                    continue
             try:
                 sm.append(float(f[1]))
                 mx.append(float(f[2]))
@@ -207,6 +218,9 @@ def main():
                                 device_id=device)
 
     w = wl.long_prefill()
+    if args.rows:
+        w = wl.Workload(f"{w.name}_rows{args.rows}", w.q[:args.rows], w.k_cache, w.v_cache,
+                        w.slot_idx[:args.rows], None)
     pairs, flops, alg_bytes, gathered = work_counts(w)
     q, k, v, idx = (x.to(device) for x in (w.q, w.k_cache, w.v_cache, w.slot_idx))
     out = torch.empty(w.Tq, w.Hq, 256, dtype=torch.bfloat16, device=device)
@@ -230,6 +244,8 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
+        time.sleep(0.3)  # let the sampler start
+        t0_epoch = time.time()
         t_wall = time.perf_counter()
         for i in range(args.steps):
             flush.zero_()
@@ -238,6 +254,7 @@ def main():
             ends[i].record(stream)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
+        t1_epoch = time.time()
     if dist is not None:
         dist.barrier()
     kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
@@ -320,7 +337,7 @@ def main():
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": alg_bytes},
         "gpu_launches": args.steps * launches_per_step,
-        "clocks": clocks.summary(),
+        "clocks": clocks.summary(t0_epoch, t1_epoch),
         "wall_s_timed_region": t_wall,
     }
     if e2e is not None:

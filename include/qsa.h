@@ -130,6 +130,46 @@ qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_str
                                 void* workspace, size_t workspace_bytes, uint32_t* err_word,
                                 void* stream);
 
+/* Size of the device scratch array that qsa_sparse_prefill_noalloc uses (16 MiB). */
+#define QSA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/*
+ * qsa_sparse_prefill_noalloc -- qsa_sparse_prefill for callers that cannot allocate.
+ *
+ * The article has no counterpart to this entry point; it exists for users of the
+ * library.  Some callers have no way to hand over a workspace: a serving runtime that
+ * reserved all free HBM for its KV-cache pool at start-up and forbids cudaMalloc
+ * afterwards, a host framework that owns the allocator and gives a plugin no hook into
+ * it, or code that must not allocate while a stream is being captured.  Only the
+ * split-W path (nsplit > 1) needs scratch; this entry point takes it from a
+ * file-scope device array of QSA_STATIC_SCRATCH_BYTES in libqsa.so, which every GPU
+ * that loads the library holds until the process exits.
+ *
+ * Arguments, layouts, ownership and errors are those of qsa_sparse_prefill without
+ * `workspace` / `workspace_bytes`.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.  Additional behaviour:
+ *   - the first call on a device (the current device) looks up that device's address
+ *     of the scratch array (cudaGetSymbolAddress) and caches it; make that first call
+ *     before any stream capture on the device;
+ *   - a shape whose plan needs more scratch than QSA_STATIC_SCRATCH_BYTES returns
+ *     QSA_ERR_WORKSPACE before any launch (qsa_sparse_prefill_plan gives the need;
+ *     a smaller nsplit request, or the workspace entry point, are the ways out);
+ *   - all calls on a device share the one array and it keeps whatever the last call
+ *     left in it; nothing in it has to start at zero (every value a call reads was
+ *     written earlier in the same call), but calls whose kernels overlap on the GPU
+ *     (e.g. on two streams) race on it: serialise them.
+ */
+qsa_status_t qsa_sparse_prefill_noalloc(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                        const void* k_cache, int64_t k_stride_s,
+                                        int64_t k_stride_h, const void* v_cache,
+                                        int64_t v_stride_s, int64_t v_stride_h,
+                                        const int32_t* slot_idx, int64_t idx_stride_t,
+                                        const int32_t* width, int32_t Tq, int32_t Hq,
+                                        int32_t Hkv, int32_t D, int64_t S, int32_t W,
+                                        float scale, void* out, int64_t out_stride_t,
+                                        int64_t out_stride_h, int32_t nsplit,
+                                        uint32_t* err_word, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 const char* qsa_status_string(qsa_status_t status);
 

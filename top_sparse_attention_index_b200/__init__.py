@@ -13,18 +13,21 @@ from ._binding import (  # noqa: F401
     QSA_ERRBIT_SLOT_RANGE,
     QSA_ERRBIT_WIDTH_RANGE,
     QSA_MAX_SLOTS_PER_SPLIT,
+    QSA_STATIC_SCRATCH_BYTES,
     QSA_OK,
     QSAError,
     load_library,
     qsa_abi_version,
     qsa_last_error_detail,
     qsa_sparse_prefill,
+    qsa_sparse_prefill_noalloc,
     qsa_sparse_prefill_plan,
     qsa_status_string,
     sparse_prefill,
 )
 
 __all__ = [
-    "sparse_prefill", "qsa_sparse_prefill", "qsa_sparse_prefill_plan", "qsa_status_string",
-    "qsa_last_error_detail", "qsa_abi_version", "load_library", "QSAError",
+    "sparse_prefill", "qsa_sparse_prefill", "qsa_sparse_prefill_noalloc",
+    "qsa_sparse_prefill_plan", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
+    "load_library", "QSAError",
 ]

@@ -22,6 +22,7 @@ QSA_ERR_CUDA = 4
 QSA_ERRBIT_SLOT_RANGE = 0x1
 QSA_ERRBIT_WIDTH_RANGE = 0x2
 QSA_MAX_SLOTS_PER_SPLIT = 2560
+QSA_STATIC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol include/qsa.h declares, with its ctypes signature (restype, argtypes).
 _p, _i32, _i64, _sz, _f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -31,6 +32,9 @@ SIGNATURES = {
     "qsa_sparse_prefill": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64, _p,
                                   _i32, _i32, _i32, _i32, _i64, _i32, _f, _p, _i64, _i64, _i32,
                                   _p, _sz, _p, _p]),
+    "qsa_sparse_prefill_noalloc": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
+                                          _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _f, _p,
+                                          _i64, _i64, _i32, _p, _p]),
     "qsa_status_string": (ctypes.c_char_p, [_i32]),
     "qsa_last_error_detail": (ctypes.c_char_p, []),
 }
@@ -97,6 +101,18 @@ def qsa_sparse_prefill(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_
         q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache, v_stride_s,
         v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W, ctypes.c_float(scale),
         out, out_stride_t, out_stride_h, nsplit, workspace, workspace_bytes, err_word, stream))
+
+
+def qsa_sparse_prefill_noalloc(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
+                               v_cache, v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq,
+                               Hq, Hkv, D, S, W, scale, out, out_stride_t, out_stride_h, nsplit,
+                               err_word, stream) -> int:
+    """Raw call of the entry point that takes its split scratch from the library's static
+    device array instead of a caller workspace; returns the status code unchanged."""
+    return int(load_library().qsa_sparse_prefill_noalloc(
+        q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache, v_stride_s,
+        v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W, ctypes.c_float(scale),
+        out, out_stride_t, out_stride_h, nsplit, err_word, stream))
 
 
 # ---- torch-facing wrapper ------------------------------------------------------------

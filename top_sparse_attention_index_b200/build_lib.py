@@ -18,7 +18,7 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 LIBRARY = PKG / "libqsa.so"
-SOURCES = [CSRC / "qsa_api.cu", CSRC / "qsa_attn.cu"]
+SOURCES = [CSRC / "qsa_api.cu", CSRC / "qsa_attn.cu", CSRC / "qsa_noalloc.cu"]
 DEPENDS = SOURCES + [CSRC / "qsa_internal.h", CSRC / "qsa_ptx.cuh", INCLUDE / "qsa.h"]
 
 NVCC_FLAGS = [

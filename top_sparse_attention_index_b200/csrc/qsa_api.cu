@@ -89,6 +89,16 @@ bool stride_ok(int64_t s) { return s >= 0 && (s % 8) == 0; }
 
 }  // namespace
 
+namespace qsa {
+// Lets other translation units of the library report a detail for their own errors.
+void set_error_detail(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+  va_end(ap);
+}
+}  // namespace qsa
+
 extern "C" {
 
 int32_t qsa_abi_version(void) { return 1; }

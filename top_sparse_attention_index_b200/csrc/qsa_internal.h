@@ -54,6 +54,9 @@ KernelShape kernel_shape(int G);
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream);
 
 size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit);
+
+// printf-style detail for qsa_last_error_detail() on the calling host thread.
+void set_error_detail(const char* fmt, ...);
 size_t workspace_lse_offset(int32_t Tq, int32_t Hq, int32_t nsplit);
 
 }  // namespace qsa

@@ -131,6 +131,7 @@ INVALID = [
     (dict(scale=float("nan")), qsa.QSA_ERR_INVALID_ARG),
     (dict(scale=float("inf")), qsa.QSA_ERR_INVALID_ARG),
     (dict(nsplit=-2), qsa.QSA_ERR_INVALID_ARG),
+    (dict(S=2 ** 30), qsa.QSA_ERR_UNSUPPORTED),           # K rows beyond 64 GiB reach
     (dict(nsplit=2, W=8, workspace=None), qsa.QSA_ERR_WORKSPACE),
     (dict(nsplit=2, W=8, workspace=0x70000, workspace_bytes=16), qsa.QSA_ERR_WORKSPACE),
 ]

@@ -36,6 +36,7 @@ constexpr int kRowBytes = kHeadDim * 2;     // one (slot, head) row: 512 bytes
 constexpr int kChunks = kRowBytes / 16;     // 32 16-byte chunks per row
 constexpr int kMergeStride = kHeadDim + 4;  // padded fp32 row of the epilogue merge
 constexpr float kNegInf = -__builtin_huge_valf();
+constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent)
 
 template <int NTILE, int SL, int STAGES>
 struct Cfg {
@@ -45,12 +46,13 @@ struct Cfg {
   static constexpr int kStageBytes = kRows * kRowBytes * 2;  // K rows then V rows
   static constexpr int kRingBytes = STAGES * kStageBytes;
   static constexpr int kQBytes = NTILE * 8 * kRowBytes;
-  static constexpr int kIdxBytes = kMaxSlotsPerSplit * 4;
+  static constexpr int kIdxBytes = kMaxSlotsPerSplit * 8;  // (K, V) row offsets per slot
   static constexpr int kScanBytes = 32 * 4;
   static constexpr int kMergeBytes = kWarps * (8 * kMergeStride + 16) * 4;
   static constexpr size_t kSmem = size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes;
   static_assert(kMergeBytes <= kRingBytes, "merge buffer reuses the ring");
-  static_assert(kIdxBytes <= kRingBytes, "raw index staging reuses the ring");
+  static_assert(kMaxSlotsPerSplit * 4 <= kRingBytes, "raw index staging reuses the ring");
+  static_assert(kMaxSlotsPerSplit % kRows == 0, "stages never read past the offset list");
   static_assert(kRows % kWarps == 0, "each warp loads whole rows");
 };
 
@@ -61,8 +63,10 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
   uint8_t* sQ = smem + C::kRingBytes;
-  int32_t* sIdx = reinterpret_cast<int32_t*>(sQ + C::kQBytes);
-  int32_t* sScan = sIdx + kMaxSlotsPerSplit;
+  // Compacted valid slots as row offsets in 16-byte units: (slot * k_stride_s / 8,
+  // slot * v_stride_s / 8); the host guarantees both fit in 32 bits.
+  uint2* sOff = reinterpret_cast<uint2*>(sQ + C::kQBytes);
+  int32_t* sScan = reinterpret_cast<int32_t*>(sOff + kMaxSlotsPerSplit);
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -127,10 +131,11 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
     int pos = warp_off + incl - cnt;
     for (int i = b_i; i < e_i; ++i) {
       const int v = sRaw[i];
-      if (v >= 0 && int64_t(v) < p.S) sIdx[pos++] = v;
+      if (v >= 0 && int64_t(v) < p.S)
+        sOff[pos++] = make_uint2(uint32_t(v) * p.k_row16, uint32_t(v) * p.v_row16);
     }
   }
-  __syncthreads();  // sIdx complete, the ring is free again
+  __syncthreads();  // sOff complete, the ring is free again
 
   const int G = p.G;
   const int64_t head0 = int64_t(j) * G;
@@ -161,9 +166,9 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
   cp_async_commit();
 
   const int n_stages = (n_valid + C::kRows - 1) / C::kRows;
-  const uint16_t* kbase = p.k_cache + int64_t(j) * p.k_stride_h;
-  const uint16_t* vbase = p.v_cache + int64_t(j) * p.v_stride_h;
-  const int ld_chunk = lane;  // each warp moves whole 512-byte rows, one chunk per lane
+  // each warp moves whole 512-byte rows, one 16-byte chunk per lane
+  const char* kbase = reinterpret_cast<const char*>(p.k_cache + int64_t(j) * p.k_stride_h) + lane * 16;
+  const char* vbase = reinterpret_cast<const char*>(p.v_cache + int64_t(j) * p.v_stride_h) + lane * 16;
 
   auto load_stage = [&](int s, int buf) {
     const uint32_t kdst = ring_s + buf * C::kStageBytes;
@@ -173,10 +178,10 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
       const int r = warp + i * C::kWarps;
       const int pos = s * C::kRows + r;
       const bool ok = pos < n_valid;
-      const int64_t slot = ok ? sIdx[pos] : 0;
-      const uint32_t off = r * kRowBytes + ((ld_chunk ^ (r & 7)) << 4);
-      cp_async_16(kdst + off, kbase + slot * p.k_stride_s + ld_chunk * 8, ok);
-      cp_async_16(vdst + off, vbase + slot * p.v_stride_s + ld_chunk * 8, ok);
+      const uint2 o = ok ? sOff[pos] : make_uint2(0u, 0u);
+      const uint32_t off = r * kRowBytes + ((lane ^ (r & 7)) << 4);
+      cp_async_16(kdst + off, kbase + size_t(o.x) * 16, ok);
+      cp_async_16(vdst + off, vbase + size_t(o.y) * 16, ok);
     }
   };
 
@@ -252,16 +257,16 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
     }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);  // finite: row `base` is valid
-    const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    const uint32_t p01 = pack_bf16x2(fast_exp2(x0 - mn0), fast_exp2(x1 - mn1));
-    const uint32_t p23 = pack_bf16x2(fast_exp2(x2 - mn0), fast_exp2(x3 - mn1));
-    // the denominators sum the same bf16-rounded weights that multiply V
-    l0 = l0 * al0 + (bf16lo_to_f32(p01) + bf16lo_to_f32(p23));
-    l1 = l1 * al1 + (bf16hi_to_f32(p01) + bf16hi_to_f32(p23));
-    if (!__all_sync(0xffffffffu, al0 == 1.f && al1 == 1.f)) {
+    // Lazy rescaling: the reference max m only moves when the chunk max exceeds it by
+    // more than kRescaleLog2 (weights stay <= 2^kRescaleLog2, exact in fp32 and within
+    // bf16 range); the final normalisation uses the same m for O and l, so the result
+    // is unchanged.  mx is finite here: row `base` of this sub-tile is valid.
+    const float mn0 = (mx0 > m0 + kRescaleLog2) ? mx0 : m0;
+    const float mn1 = (mx1 > m1 + kRescaleLog2) ? mx1 : m1;
+    if (__any_sync(0xffffffffu, mn0 != m0 || mn1 != m1)) {
+      const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);  // -inf -> 0
+      l0 *= al0;
+      l1 *= al1;
 #pragma unroll
       for (int mt = 0; mt < 16; ++mt) {
         o[mt][0] *= al0;
@@ -269,7 +274,14 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
         o[mt][2] *= al0;
         o[mt][3] *= al1;
       }
+      m0 = mn0;
+      m1 = mn1;
     }
+    const uint32_t p01 = pack_bf16x2(fast_exp2(x0 - m0), fast_exp2(x1 - m1));
+    const uint32_t p23 = pack_bf16x2(fast_exp2(x2 - m0), fast_exp2(x3 - m1));
+    // the denominators sum the same bf16-rounded weights that multiply V
+    l0 += bf16lo_to_f32(p01) + bf16lo_to_f32(p23);
+    l1 += bf16hi_to_f32(p01) + bf16hi_to_f32(p23);
 
     // O^T (256 x 8) += V^T (256 x 16) * P^T (16 x 8)
     const uint32_t b0 = movmatrix_trans(p01);

@@ -34,6 +34,8 @@ struct FwdParams {
   int32_t Tq, Hq, Hkv, G, W;
   int32_t nsplit;
   int32_t split_len;        // positions of the W axis per split
+  uint32_t k_row16;         // k_stride_s / 8: one slot step of K in 16-byte units
+  uint32_t v_row16;         // v_stride_s / 8
   float scale_log2;         // scale * log2(e)
 };
 

@@ -50,7 +50,10 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--rows", type=int, default=0,
-                    help="keep only the first ROWS query rows (small cases for ncu captures)")
+                    help="keep only the first ROWS query rows (small cases for ncu captures, "
+                         "decode-like batches)")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of a CUDA graph that holds one step")
     return ap.parse_args()
 
 
@@ -237,6 +240,15 @@ def main():
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        step = graph.replay
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
 
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -328,7 +340,8 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.name, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": 256, "S": w.S,
                    "W": w.W, "valid_pairs": pairs, "nsplit": nsplit,
-                   "l2": "flushed between steps (512 MiB write)", "parallelism": f"replicas x{world}"},
+                   "l2": "flushed between steps (512 MiB write)", "parallelism": f"replicas x{world}",
+                   "launch": "cuda graph replay" if args.graph else "eager"},
         "pairs_per_s": world * pairs / t_s,
         "pairs_x_hkv_per_s": world * pairs * w.Hkv / t_s,
         "gathered_gb_per_s": gathered / t_s / 1e9,

@@ -319,3 +319,48 @@ def test_invalid_arguments_with_device_tensors(cuda_device):
     assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert (out == 3.0).all()   # nothing was launched
+
+
+# ---- decode-like batches under CUDA graph capture -------------------------------------
+
+def _raw_call(d, out, ws, nsplit, stream):
+    q, k, v, idx = d["q"], d["k_cache"], d["v_cache"], d["slot_idx"]
+    return qsa.qsa_sparse_prefill(
+        q.data_ptr(), q.stride(0), q.stride(1), k.data_ptr(), k.stride(0), k.stride(1),
+        v.data_ptr(), v.stride(0), v.stride(1), idx.data_ptr(), idx.stride(0),
+        None if d["width"] is None else d["width"].data_ptr(), q.shape[0], q.shape[1], k.shape[1],
+        D, k.shape[0], idx.shape[1], 1.0 / 16.0, out.data_ptr(), out.stride(0), out.stride(1),
+        nsplit, None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(), None,
+        stream)
+
+
+@pytest.mark.parametrize("Tq", [1, 8, 64])
+def test_cuda_graph_capture_decode_shape(cuda_device, oracle_lib, Tq):
+    """Few query rows with a wide selection (all parallelism from split-W plus the
+    combine kernel).  The call only enqueues kernels on the given stream, so it can be
+    captured into a CUDA graph; replays on new inputs written into the same buffers
+    match the oracle."""
+    cases = [_random_case(900 + Tq + i, Tq, 16, 2, 65536, 2051, minus1=0.1, widths=True)
+             for i in range(2)]
+    d = dev(cases[0], cuda_device)
+    num_sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    nsplit, ws_bytes = qsa.qsa_sparse_prefill_plan(Tq, 16, 2, D, 2051, num_sms)
+    assert nsplit > 1
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=cuda_device)
+    out = torch.empty(Tq, 16, D, dtype=torch.bfloat16, device=cuda_device)
+    # one eager call first: it sets the kernels' per-device attributes
+    assert _raw_call(d, out, ws, nsplit, torch.cuda.current_stream().cuda_stream) == qsa.QSA_OK
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st = _raw_call(d, out, ws, nsplit, torch.cuda.current_stream().cuda_stream)
+    assert st == qsa.QSA_OK
+    for w in cases:
+        for key, src in (("q", w.q), ("k_cache", w.k_cache), ("v_cache", w.v_cache),
+                         ("slot_idx", w.slot_idx), ("width", w.width)):
+            d[key].copy_(src)
+        out.fill_(7.0)
+        g.replay()
+        torch.cuda.synchronize()
+        ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0)
+        check_gates(out.cpu().float(), torch.from_numpy(ref), empty_rows(w), f"graph Tq={Tq}")

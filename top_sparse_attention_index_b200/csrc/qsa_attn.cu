@@ -9,9 +9,12 @@
 // K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit:
 //   1. stage the split's slot indices in shared memory and compact away -1 (and
 //      out-of-range) entries with a block scan, so masked slots cost no bandwidth;
-//   2. gather K and V rows of the compacted slots with 16-byte cp.async into a
-//      STAGES-deep shared-memory ring (row = 512 contiguous bytes; the 16-byte chunks
-//      of a row are XOR-swizzled by the row index so ldmatrix reads are conflict-free);
+//   2. gather K and V rows of the compacted slots with 16-byte cp.async into shared
+//      memory: each 16-slot sub-tile of a stage belongs to one slot lane (one warp, or a
+//      warp pair when G > 8) that loads it, waits for it and consumes it, so the lanes
+//      run STAGES-deep pipelines of their own with no block-wide barrier in the loop
+//      (row = 512 contiguous bytes; the 16-byte chunks of a row are XOR-swizzled by the
+//      row index so ldmatrix reads are conflict-free);
 //   3. per warp and 16-slot sub-tile: S^T = K Q^T with the slots as the MMA M dimension
 //      and the (up to 8) heads of one n8 tile as N, so the group shares every gathered
 //      row and G = 3/6/8/12/16 needs no padding of the head ratio in memory;
@@ -24,6 +27,7 @@
 //   split partials; empty splits carry LSE = -inf and weight 0; all empty -> exact 0.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "qsa_internal.h"
@@ -38,13 +42,15 @@ constexpr int kMergeStride = kHeadDim + 4;  // padded fp32 row of the epilogue m
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent)
 
+
 template <int NTILE, int SL, int STAGES>
 struct Cfg {
   static constexpr int kWarps = NTILE * SL;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kRows = 16 * SL;                      // slots per stage
-  static constexpr int kStageBytes = kRows * kRowBytes * 2;  // K rows then V rows
-  static constexpr int kRingBytes = STAGES * kStageBytes;
+  static constexpr int kSubBytes = 16 * kRowBytes * 2;       // one sub-tile: 16 K rows, 16 V rows
+  static constexpr int kStageBytes = SL * kSubBytes;
+  static constexpr int kRingBytes = STAGES * kStageBytes;    // [slot lane][stage][sub-tile]
   static constexpr int kQBytes = NTILE * 8 * kRowBytes;
   static constexpr int kIdxBytes = kMaxSlotsPerSplit * 8;  // (K, V) row offsets per slot
   static constexpr int kScanBytes = 32 * 4;
@@ -52,8 +58,7 @@ struct Cfg {
   static constexpr size_t kSmem = size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes;
   static_assert(kMergeBytes <= kRingBytes, "merge buffer reuses the ring");
   static_assert(kMaxSlotsPerSplit * 4 <= kRingBytes, "raw index staging reuses the ring");
-  static_assert(kMaxSlotsPerSplit % kRows == 0, "stages never read past the offset list");
-  static_assert(kRows % kWarps == 0, "each warp loads whole rows");
+  static_assert(kMaxSlotsPerSplit % 16 == 0, "the offset list pads to whole sub-tiles");
 };
 
 template <int NTILE, int SL, int STAGES>
@@ -166,24 +171,42 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
   cp_async_commit();
 
   const int n_stages = (n_valid + C::kRows - 1) / C::kRows;
-  // each warp moves whole 512-byte rows, one 16-byte chunk per lane
+  // Pad the offset list to whole 16-slot sub-tiles with the first slot: padding rows
+  // hold finite data and are masked out of the softmax.
+  for (int i = n_valid + tid; i < ((n_valid + 15) & ~15); i += C::kThreads) sOff[i] = sOff[0];
   const char* kbase = reinterpret_cast<const char*>(p.k_cache + int64_t(j) * p.k_stride_h) + lane * 16;
   const char* vbase = reinterpret_cast<const char*>(p.v_cache + int64_t(j) * p.v_stride_h) + lane * 16;
+  const uint32_t lane16 = uint32_t(lane) << 4;
+  // this lane's sub-tiles: [wslot][stage]; a warp pair splits the 16 rows 8 / 8
+  const uint32_t sub_s = ring_s + wslot * STAGES * C::kSubBytes;
+  constexpr int kLoadRows = 16 / NTILE;
+  const int row0 = wn * kLoadRows;
 
   auto load_stage = [&](int s, int buf) {
-    const uint32_t kdst = ring_s + buf * C::kStageBytes;
-    const uint32_t vdst = kdst + C::kRows * kRowBytes;
+    const int base = s * C::kRows + wslot * 16;
+    if (base >= n_valid) return;  // an empty sub-tile is neither loaded nor read
+    const uint32_t kdst = sub_s + buf * C::kSubBytes;
 #pragma unroll
-    for (int i = 0; i < C::kRows / C::kWarps; ++i) {
-      const int r = warp + i * C::kWarps;
-      const int pos = s * C::kRows + r;
-      const bool ok = pos < n_valid;
-      const uint2 o = ok ? sOff[pos] : make_uint2(0u, 0u);
-      const uint32_t off = r * kRowBytes + ((lane ^ (r & 7)) << 4);
-      cp_async_16(kdst + off, kbase + size_t(o.x) * 16, ok);
-      cp_async_16(vdst + off, vbase + size_t(o.y) * 16, ok);
+    for (int i = 0; i < kLoadRows; i += 2) {
+      const uint4 o2 = *reinterpret_cast<const uint4*>(sOff + base + row0 + i);  // rows r, r+1
+      const int r = row0 + i;
+      const uint32_t d0 = kdst + r * kRowBytes + (lane16 ^ ((r & 7) << 4));
+      const uint32_t d1 = kdst + (r + 1) * kRowBytes + (lane16 ^ (((r + 1) & 7) << 4));
+      cp_async_16(d0, kbase + size_t(o2.x) * 16);
+      cp_async_16(d0 + 16 * kRowBytes, vbase + size_t(o2.y) * 16);
+      cp_async_16(d1, kbase + size_t(o2.z) * 16);
+      cp_async_16(d1 + 16 * kRowBytes, vbase + size_t(o2.w) * 16);
     }
   };
+  // makes a stage's sub-tile, loaded by one warp or a warp pair, visible to it
+  auto lane_sync = [&]() {
+    if constexpr (NTILE == 1) {
+      __syncwarp();
+    } else {
+      named_barrier_sync(1 + wslot, 32 * NTILE);
+    }
+  };
+  __syncthreads();  // the padded offset list is complete
 
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
@@ -208,22 +231,22 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
   }
 
   // ---- 3. main loop ------------------------------------------------------------------
-  float m0 = kNegInf, m1 = kNegInf;  // running max (base 2) of heads 2(l%4), 2(l%4)+1
+  float m0 = kNegInf, m1 = kNegInf;  // reference max (base 2) of heads 2(l%4), 2(l%4)+1
   float l0 = 0.f, l1 = 0.f;          // this lane's share of the running sums
   float o[16][4];
 #pragma unroll
   for (int mt = 0; mt < 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
   const int key = lane & 7;  // swizzle key of every row this lane addresses
-  const int krow = wslot * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int krow = (lane & 7) + ((lane >> 3) & 1) * 8;
   const int khi = lane >> 4;
-  const int vrow = wslot * 16 + (lane & 7) + ((lane >> 4) << 3);
+  const int vrow = (lane & 7) + ((lane >> 4) << 3);
   const int vhi = (lane >> 3) & 1;
   const float sl2 = p.scale_log2;
 
   for (int s = 0; s < n_stages; ++s) {
     cp_async_wait<STAGES - 2>();
-    __syncthreads();
+    lane_sync();  // stage s landed for the whole slot lane; stage s-1 is consumed
     {
       const int sn = s + STAGES - 1;
       if (sn < n_stages) load_stage(sn, sn % STAGES);
@@ -232,9 +255,10 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
     const int buf = s % STAGES;
     const int base = s * C::kRows + wslot * 16;
     if (base >= n_valid) continue;  // warp-uniform: no valid slot in this sub-tile
+    const uint32_t sub = sub_s + buf * C::kSubBytes;
 
     // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8); two chains for ILP.
-    const uint32_t kt = ring_s + buf * C::kStageBytes + krow * kRowBytes;
+    const uint32_t kt = sub + krow * kRowBytes;
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 16; ks += 2) {
@@ -286,7 +310,7 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
     // O^T (256 x 8) += V^T (256 x 16) * P^T (16 x 8)
     const uint32_t b0 = movmatrix_trans(p01);
     const uint32_t b1 = movmatrix_trans(p23);
-    const uint32_t vt = ring_s + buf * C::kStageBytes + C::kRows * kRowBytes + vrow * kRowBytes;
+    const uint32_t vt = sub + 16 * kRowBytes + vrow * kRowBytes;
 #pragma unroll
     for (int mt = 0; mt < 16; ++mt) {
       uint32_t a[4];
@@ -409,24 +433,49 @@ template <int NTILE, int SL, int STAGES>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
   using C = Cfg<NTILE, SL, STAGES>;
   auto kern = qsa_sparse_attn_fwd_kernel<NTILE, SL, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(C::kSmem));
+  // The shared-memory opt-in is a per-device function attribute: set it on the first
+  // launch on each device only, so later calls (e.g. under stream capture) are launches
+  // and nothing else.
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit == 0 || !(configured.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(C::kSmem));
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
   const unsigned grid = static_cast<unsigned>(int64_t(p.Tq) * p.Hkv * p.nsplit);
   kern<<<grid, C::kThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError();
 }
 
-// The two shapes: G <= 8 (one n8 tile, 4 slot lanes, 64-slot stages, 3 stages) and
-// 8 < G <= 16 (two n8 tiles, 2 slot lanes, 32-slot stages, 6 stages).
-using CfgSmall = Cfg<1, 4, 3>;
-using CfgLarge = Cfg<2, 2, 6>;
+// The two shapes (slot lanes x pipeline stages per lane, chosen by measurement):
+// G <= 8: one n8 tile, QSA_SMALL_SL slot lanes of one warp each;
+// 8 < G <= 16: two n8 tiles, QSA_LARGE_SL slot lanes of a warp pair each.
+#ifndef QSA_SMALL_SL
+#define QSA_SMALL_SL 6
+#endif
+#ifndef QSA_SMALL_STAGES
+#define QSA_SMALL_STAGES 2
+#endif
+#ifndef QSA_LARGE_SL
+#define QSA_LARGE_SL 6
+#endif
+#ifndef QSA_LARGE_STAGES
+#define QSA_LARGE_STAGES 2
+#endif
+using CfgSmall = Cfg<1, QSA_SMALL_SL, QSA_SMALL_STAGES>;
+using CfgLarge = Cfg<2, QSA_LARGE_SL, QSA_LARGE_STAGES>;
 
 }  // namespace
 
 KernelShape kernel_shape(int G) {
-  if (G <= 8) return {1, 4, CfgSmall::kThreads, CfgSmall::kRows, 3, CfgSmall::kSmem, 1};
-  return {2, 2, CfgLarge::kThreads, CfgLarge::kRows, 6, CfgLarge::kSmem, 1};
+  if (G <= 8)
+    return {1, QSA_SMALL_SL, CfgSmall::kThreads, CfgSmall::kRows, QSA_SMALL_STAGES, CfgSmall::kSmem, 1};
+  return {2, QSA_LARGE_SL, CfgLarge::kThreads, CfgLarge::kRows, QSA_LARGE_STAGES, CfgLarge::kSmem, 1};
 }
 
 size_t workspace_lse_offset(int32_t Tq, int32_t Hq, int32_t nsplit) {
@@ -441,7 +490,8 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
 }
 
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = (p.G <= 8) ? launch_fwd<1, 4, 3>(p, stream) : launch_fwd<2, 2, 6>(p, stream);
+  cudaError_t e = (p.G <= 8) ? launch_fwd<1, QSA_SMALL_SL, QSA_SMALL_STAGES>(p, stream)
+                             : launch_fwd<2, QSA_LARGE_SL, QSA_LARGE_STAGES>(p, stream);
   if (e != cudaSuccess || p.nsplit == 1) return e;
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);

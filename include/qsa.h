@@ -130,6 +130,38 @@ qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_str
                                 void* workspace, size_t workspace_bytes, uint32_t* err_word,
                                 void* stream);
 
+/* Largest block size of block selection. */
+#define QSA_MAX_BLOCK 16
+
+/*
+ * qsa_sparse_prefill_block_plan / qsa_sparse_prefill_block -- block selection.
+ *
+ * Source: the article "Qwen4-Exp QSA comes to Huawei's Ascend: inside SGLang's opt-in
+ * CANN prefill PR", section "Why QSA is the awkward part, in numbers": the indexer
+ * selects micro-blocks (compression ratio 4, a budget of 2,048 micro-blocks per query);
+ * the article's path keeps sparse block size 1 and names "block4" as later work.
+ * Reading taken here: every selected entry b of slot_idx names the `block` consecutive
+ * physical slots b*block .. b*block + block - 1 (block 4 = micro-blocks of four tokens
+ * laid out contiguously in the cache).  An entry is valid when it is not -1 and its
+ * whole block lies in [0, S); any other value is masked and sets QSA_ERRBIT_SLOT_RANGE.
+ * W counts entries (blocks).  1 <= block <= QSA_MAX_BLOCK (QSA_ERR_INVALID_ARG
+ * otherwise).  Everything else is exactly qsa_sparse_prefill_plan / qsa_sparse_prefill,
+ * which are these functions with block = 1.
+ */
+int32_t qsa_sparse_prefill_block_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W,
+                                      int32_t block, int32_t num_sms, int32_t nsplit_request,
+                                      size_t* workspace_bytes);
+
+qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                      const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                      const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                      const int32_t* slot_idx, int64_t idx_stride_t,
+                                      const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                      int32_t D, int64_t S, int32_t W, int32_t block, float scale,
+                                      void* out, int64_t out_stride_t, int64_t out_stride_h,
+                                      int32_t nsplit, void* workspace, size_t workspace_bytes,
+                                      uint32_t* err_word, void* stream);
+
 /* Size of the device scratch array that qsa_sparse_prefill_noalloc uses (16 MiB). */
 #define QSA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 

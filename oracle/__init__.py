@@ -49,6 +49,10 @@ class Oracle:
         p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
         f.argtypes = [p, i64, i64, p, i64, i64, p, i64, i64, p, i64, p,
                       i32, i32, i32, i32, i64, i32, ctypes.c_float, p, i64, p, p]
+        fb = self._lib.qsa_oracle_forward_block
+        fb.restype = ctypes.c_int
+        fb.argtypes = [p, i64, i64, p, i64, i64, p, i64, i64, p, i64, p,
+                       i32, i32, i32, i32, i64, i32, i32, ctypes.c_float, p, i64, p, p]
         self._lib.qsa_oracle_num_threads.restype = ctypes.c_int
         self.path = path
 
@@ -56,13 +60,14 @@ class Oracle:
         return int(self._lib.qsa_oracle_num_threads())
 
     def forward(self, q, k_cache, v_cache, slot_idx, width=None, scale=1.0 / 16.0, rows=None,
-                S=None, return_err=False):
+                S=None, return_err=False, block=1):
         """fp32 oracle output for query rows ``rows`` (all rows when None).
 
         q: bf16 bits as uint16 array [Tq, Hq, D] (any strides, d contiguous) or a torch
         bf16 CPU tensor; k_cache / v_cache: [S, Hkv, D] likewise; slot_idx: int32
         [Tq, W] (row-strided, column-contiguous); width: int32 [Tq] or None.
         Returns float32 [len(rows) or Tq, Hq, D] (and the error bits when asked).
+        With block > 1 every entry of slot_idx names `block` consecutive slots.
         """
         q, k_cache, v_cache = (_as_bf16_bits(x) for x in (q, k_cache, v_cache))
         slot_idx = _as_i32(slot_idx)
@@ -84,15 +89,17 @@ class Oracle:
             nrows = Tq
         out = np.zeros((nrows, Hq, D), dtype=np.float32)
         err = ctypes.c_uint32(0)
-        rc = self._lib.qsa_oracle_forward(
-            q.ctypes.data, q.strides[0] // 2, q.strides[1] // 2,
-            k_cache.ctypes.data, k_cache.strides[0] // 2, k_cache.strides[1] // 2,
-            v_cache.ctypes.data, v_cache.strides[0] // 2, v_cache.strides[1] // 2,
-            slot_idx.ctypes.data, slot_idx.strides[0] // 4,
-            None if width is None else width.ctypes.data,
-            Tq, Hq, Hkv, D, S, W, ctypes.c_float(scale),
-            None if rows is None else rows.ctypes.data, nrows,
-            out.ctypes.data, ctypes.byref(err))
+        common = (q.ctypes.data, q.strides[0] // 2, q.strides[1] // 2,
+                  k_cache.ctypes.data, k_cache.strides[0] // 2, k_cache.strides[1] // 2,
+                  v_cache.ctypes.data, v_cache.strides[0] // 2, v_cache.strides[1] // 2,
+                  slot_idx.ctypes.data, slot_idx.strides[0] // 4,
+                  None if width is None else width.ctypes.data, Tq, Hq, Hkv, D, S, W)
+        tail = (ctypes.c_float(scale), None if rows is None else rows.ctypes.data, nrows,
+                out.ctypes.data, ctypes.byref(err))
+        if block == 1:
+            rc = self._lib.qsa_oracle_forward(*common, *tail)
+        else:
+            rc = self._lib.qsa_oracle_forward_block(*common, block, *tail)
         if rc != 0:
             raise ValueError("oracle rejected the sizes")
         return (out, int(err.value)) if return_err else out

@@ -150,6 +150,73 @@ int qsa_oracle_forward(const uint16_t* q, int64_t q_stride_t, int64_t q_stride_h
   return 0;
 }
 
+/*
+ * qsa_oracle_forward_block -- block selection: every selected entry b of slot_idx names
+ * the `block` consecutive physical slots b*block .. b*block + block - 1 (sparse block
+ * size `block`; the article's path keeps block size 1 and names "block4" as later work,
+ * section "Why QSA is the awkward part, in numbers").  The definition: expand each
+ * valid entry into its slots, in order, then apply the slot-level definition above.
+ * An entry is valid when it is not -1 and its whole block lies in [0, S); any other
+ * value raises bit 0 of *err_bits and is skipped.  Arguments as qsa_oracle_forward,
+ * W counting entries (blocks), plus `block` >= 1.
+ */
+int qsa_oracle_forward_block(const uint16_t* q, int64_t q_stride_t, int64_t q_stride_h,
+                             const uint16_t* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                             const uint16_t* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                             const int32_t* slot_idx, int64_t idx_stride_t, const int32_t* width,
+                             int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int64_t S, int32_t W,
+                             int32_t block, float scale, const int64_t* rows, int64_t nrows,
+                             float* out, uint32_t* err_bits) {
+  if (Tq < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || S < 0 || W < 0 || block < 1) return -1;
+  if (Hq % Hkv != 0) return -1;
+  const int32_t G = Hq / Hkv;
+  const int64_t n_out = rows ? nrows : (int64_t)Tq;
+  const int64_t cap = (int64_t)W * block;
+  uint32_t all_bits = 0;
+
+#pragma omp parallel reduction(| : all_bits)
+  {
+    int32_t* expanded = (int32_t*)malloc(sizeof(int32_t) * (size_t)(cap > 0 ? cap : 1));
+    float* scratch_s = (float*)malloc(sizeof(float) * (size_t)(cap > 0 ? cap : 1));
+    int64_t* scratch_i = (int64_t*)malloc(sizeof(int64_t) * (size_t)(cap > 0 ? cap : 1));
+    uint32_t bits = 0;
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_out; ++r) {
+      const int64_t t = rows ? rows[r] : r;
+      int32_t width_t = width ? width[t] : W;
+      if (width_t < 0 || width_t > W) {
+        bits |= 2u;
+        width_t = width_t < 0 ? 0 : W;
+      }
+      /* expand the valid blocks into their slots */
+      const int32_t* idx_row = slot_idx + t * idx_stride_t;
+      int32_t n = 0;
+      for (int32_t w = 0; w < width_t; ++w) {
+        const int32_t b = idx_row[w];
+        if (b == -1) continue;
+        if (b < -1 || ((int64_t)b + 1) * block > S) {
+          bits |= 1u;
+          continue;
+        }
+        for (int32_t e = 0; e < block; ++e) expanded[n++] = b * block + e;
+      }
+      for (int32_t h = 0; h < Hq; ++h) {
+        const int32_t j = h / G;
+        const uint16_t* q_row = q + t * q_stride_t + (int64_t)h * q_stride_h;
+        float* out_row = out + (r * Hq + h) * (int64_t)D;
+        oracle_row(q_row, k_cache, v_cache, k_stride_s, k_stride_h, v_stride_s, v_stride_h,
+                   expanded, n, j, D, S, scale, out_row, scratch_s, scratch_i, &bits);
+      }
+    }
+    free(expanded);
+    free(scratch_s);
+    free(scratch_i);
+    all_bits |= bits;
+  }
+  if (err_bits) *err_bits |= all_bits;
+  return 0;
+}
+
 /* Number of OpenMP threads a parallel region of this library uses (1 without OpenMP). */
 int qsa_oracle_num_threads(void) {
 #ifdef _OPENMP

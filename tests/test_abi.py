@@ -73,6 +73,18 @@ def test_plan_splits_small_batches(lib):
     assert -(-2051 // n1) >= 128
 
 
+def test_block_plan(lib):
+    # 2,048 blocks of 4 = 8,192 slots per row: at least ceil(8192 / 2560) = 4 splits
+    n, ws = qsa.qsa_sparse_prefill_block_plan(7810, 16, 2, 256, 2048, 4, 148)
+    assert n == 4 and ws > 0
+    assert qsa.qsa_sparse_prefill_block_plan(7810, 16, 2, 256, 2051, 1, 148) == \
+        qsa.qsa_sparse_prefill_plan(7810, 16, 2, 256, 2051, 148)
+    for bad in (0, 17, -4):
+        with pytest.raises(qsa.QSAError) as ei:
+            qsa.qsa_sparse_prefill_block_plan(10, 16, 2, 256, 8, bad, 148)
+        assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+
+
 def test_plan_wide_rows_force_splits(lib):
     n, _ = qsa.qsa_sparse_prefill_plan(100000, 16, 2, 256, 6000, 148)
     assert n == 3  # ceil(6000 / 2560)

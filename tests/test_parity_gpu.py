@@ -364,3 +364,62 @@ def test_cuda_graph_capture_decode_shape(cuda_device, oracle_lib, Tq):
         torch.cuda.synchronize()
         ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0)
         check_gates(out.cpu().float(), torch.from_numpy(ref), empty_rows(w), f"graph Tq={Tq}")
+
+
+# ---- block selection -------------------------------------------------------------------
+
+def _block_case(seed, Tq, Hq, Hkv, S, Wb, block, minus1=0.1, widths=True):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(Tq, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    idx = wl.uniform_distinct(g, Tq, S // block, Wb)
+    if minus1:
+        idx[torch.rand(Tq, Wb, generator=g) < minus1] = -1
+    width = torch.randint(0, Wb + 1, (Tq,), generator=g, dtype=torch.int32) if widths else None
+    return wl.Workload(f"block{block}_{Tq}", q, k, v, idx, width)
+
+
+@pytest.mark.parametrize("block,Hq,Hkv", [(4, 16, 2), (2, 24, 2), (4, 6, 1), (16, 16, 2)])
+@pytest.mark.parametrize("nsplit", [0, 3])
+def test_block_selection(cuda_device, oracle_lib, block, Hq, Hkv, nsplit):
+    """Each entry names `block` consecutive slots (block 4: micro-blocks of four tokens)."""
+    w = _block_case(300 + block + Hq, 129, Hq, Hkv, 16384, 2048 // block, block)
+    d = dev(w, cuda_device)
+    out = qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"], d["width"],
+                             scale=1.0 / 16.0, nsplit=nsplit, block=block)
+    torch.cuda.synchronize()
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0, block=block)
+    cnt = valid_counts(w.slot_idx, w.width, w.S // block)
+    check_gates(out.cpu().float(), torch.from_numpy(ref), (cnt == 0).nonzero().flatten().tolist(),
+                f"block {block}")
+
+
+def test_block4_budget_rows(cuda_device, oracle_lib):
+    """The indexer's budget of 2,048 micro-blocks of 4 slots: 8,192 slots per query row,
+    more than one split can hold, over the 65,536-slot long-prefill cache."""
+    w = _block_case(310, 512, 16, 2, 65536, 2048, 4, minus1=0.0, widths=False)
+    n, _ = qsa.qsa_sparse_prefill_block_plan(512, 16, 2, D, 2048, 4, 148)
+    assert n >= 4
+    d = dev(w, cuda_device)
+    out = qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"], block=4)
+    torch.cuda.synchronize()
+    rows = list(range(0, 512, 9))
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0, rows=rows, block=4)
+    check_gates(out.cpu()[rows].float(), torch.from_numpy(ref), None, "block4 budget")
+
+
+def test_block_past_cache_end_is_flagged(cuda_device, oracle_lib):
+    w = _block_case(320, 16, 16, 2, 1000, 40, 4, minus1=0.0, widths=False)
+    w.slot_idx[2, 5] = 250          # slots 1000..1003: past S = 1000
+    w.slot_idx[4, 0] = -3
+    d = dev(w, cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"], block=4,
+                             err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & qsa.QSA_ERRBIT_SLOT_RANGE
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0, block=4)
+    check_gates(out.cpu().float(), torch.from_numpy(ref), None, "block past end")
+    with pytest.raises(qsa.QSAError):
+        qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"], block=17)

@@ -12,6 +12,7 @@ from ._binding import (  # noqa: F401
     QSA_ERR_WORKSPACE,
     QSA_ERRBIT_SLOT_RANGE,
     QSA_ERRBIT_WIDTH_RANGE,
+    QSA_MAX_BLOCK,
     QSA_MAX_SLOTS_PER_SPLIT,
     QSA_STATIC_SCRATCH_BYTES,
     QSA_OK,
@@ -20,6 +21,8 @@ from ._binding import (  # noqa: F401
     qsa_abi_version,
     qsa_last_error_detail,
     qsa_sparse_prefill,
+    qsa_sparse_prefill_block,
+    qsa_sparse_prefill_block_plan,
     qsa_sparse_prefill_noalloc,
     qsa_sparse_prefill_plan,
     qsa_status_string,
@@ -28,6 +31,7 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "sparse_prefill", "qsa_sparse_prefill", "qsa_sparse_prefill_noalloc",
+    "qsa_sparse_prefill_block", "qsa_sparse_prefill_block_plan",
     "qsa_sparse_prefill_plan", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
     "load_library", "QSAError",
 ]

@@ -22,6 +22,7 @@ QSA_ERR_CUDA = 4
 QSA_ERRBIT_SLOT_RANGE = 0x1
 QSA_ERRBIT_WIDTH_RANGE = 0x2
 QSA_MAX_SLOTS_PER_SPLIT = 2560
+QSA_MAX_BLOCK = 16
 QSA_STATIC_SCRATCH_BYTES = 16 << 20
 
 # Every symbol include/qsa.h declares, with its ctypes signature (restype, argtypes).
@@ -32,6 +33,11 @@ SIGNATURES = {
     "qsa_sparse_prefill": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64, _p,
                                   _i32, _i32, _i32, _i32, _i64, _i32, _f, _p, _i64, _i64, _i32,
                                   _p, _sz, _p, _p]),
+    "qsa_sparse_prefill_block_plan": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                             ctypes.POINTER(_sz)]),
+    "qsa_sparse_prefill_block": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64,
+                                        _p, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _f, _p, _i64,
+                                        _i64, _i32, _p, _sz, _p, _p]),
     "qsa_sparse_prefill_noalloc": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _f, _p,
                                           _i64, _i64, _i32, _p, _p]),
@@ -103,6 +109,28 @@ def qsa_sparse_prefill(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_
         out, out_stride_t, out_stride_h, nsplit, workspace, workspace_bytes, err_word, stream))
 
 
+def qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, block, num_sms, nsplit_request=0):
+    """(nsplit, workspace_bytes) for block selection; raises QSAError for invalid shapes."""
+    ws = ctypes.c_size_t(0)
+    n = int(load_library().qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, block, num_sms,
+                                                         nsplit_request, ctypes.byref(ws)))
+    if n < 0:
+        raise QSAError(-n, qsa_last_error_detail())
+    return n, int(ws.value)
+
+
+def qsa_sparse_prefill_block(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,
+                             v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv,
+                             D, S, W, block, scale, out, out_stride_t, out_stride_h, nsplit,
+                             workspace, workspace_bytes, err_word, stream) -> int:
+    """Raw call of block selection (each entry names `block` consecutive slots)."""
+    return int(load_library().qsa_sparse_prefill_block(
+        q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache, v_stride_s,
+        v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W, block,
+        ctypes.c_float(scale), out, out_stride_t, out_stride_h, nsplit, workspace,
+        workspace_bytes, err_word, stream))
+
+
 def qsa_sparse_prefill_noalloc(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
                                v_cache, v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq,
                                Hq, Hkv, D, S, W, scale, out, out_stride_t, out_stride_h, nsplit,
@@ -131,13 +159,14 @@ def _check_dev(name, t, dtype, device):
 
 
 def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=None, nsplit=0,
-                   err_word=None, stream=None):
+                   err_word=None, stream=None, block=1):
     """Selected-slot sparse attention on the GPU.
 
     q [Tq, Hq, 256] bf16, k_cache / v_cache [S, Hkv, 256] bf16, slot_idx [Tq, W] int32
     (-1 = masked), width [Tq] int32 or None; scale defaults to 1/sqrt(256) = 1/16.
     Returns out [Tq, Hq, 256] bf16 (allocated unless given).  Work is enqueued on
-    ``stream`` (default: torch's current stream); nothing is synchronised.
+    ``stream`` (default: torch's current stream); nothing is synchronised.  With
+    block > 1 every entry of slot_idx names `block` consecutive slots.
     """
     device = q.device
     if device.type != "cuda":
@@ -167,13 +196,13 @@ def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=No
     if stream is None:
         stream = torch.cuda.current_stream(device)
     num_sms = torch.cuda.get_device_properties(device).multi_processor_count
-    ns, ws_bytes = qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms, nsplit)
+    ns, ws_bytes = qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, block, num_sms, nsplit)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device) if ws_bytes else None
     with torch.cuda.device(device):
-        st = qsa_sparse_prefill(
+        st = qsa_sparse_prefill_block(
             _ptr(q), q.stride(0), q.stride(1), _ptr(k_cache), k_cache.stride(0), k_cache.stride(1),
             _ptr(v_cache), v_cache.stride(0), v_cache.stride(1), _ptr(slot_idx) if W else None,
-            slot_idx.stride(0), _ptr(width), Tq, Hq, Hkv, D, S, W, float(scale), _ptr(out),
+            slot_idx.stride(0), _ptr(width), Tq, Hq, Hkv, D, S, W, block, float(scale), _ptr(out),
             out.stride(0), out.stride(1), ns, _ptr(ws), ws_bytes, _ptr(err_word), stream.cuda_stream)
     if st != QSA_OK:
         raise QSAError(st, qsa_last_error_detail())

@@ -35,6 +35,12 @@ struct Plan {
 };
 
 // Shape validation shared by the planner and the launch; returns QSA_OK or an error.
+qsa_status_t check_block(int32_t block) {
+  if (block < 1 || block > qsa::kMaxBlock)
+    return fail(QSA_ERR_INVALID_ARG, "block size %d outside 1..%d", block, qsa::kMaxBlock);
+  return QSA_OK;
+}
+
 qsa_status_t check_shape(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W) {
   if (Tq < 0 || W < 0) return fail(QSA_ERR_INVALID_ARG, "negative size: Tq=%d W=%d", Tq, W);
   if (Hq <= 0 || Hkv <= 0 || D <= 0)
@@ -46,9 +52,14 @@ qsa_status_t check_shape(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t
   return QSA_OK;
 }
 
-Plan make_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W, int32_t num_sms, int32_t request) {
+// Splits of the W axis.  One split's slots (entries x block) must fit the shared-memory
+// offset list; with few work units, more splits fill about two waves of CTAs but none
+// is narrower than kMinSlotsPerSplit slots.
+Plan make_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W, int32_t block, int32_t num_sms,
+               int32_t request) {
   const int32_t G = Hq / Hkv;
-  const int32_t min_split = W > 0 ? (W + qsa::kMaxSlotsPerSplit - 1) / qsa::kMaxSlotsPerSplit : 1;
+  const int32_t per_split_max = qsa::kMaxSlotsPerSplit / block;  // entries
+  const int32_t min_split = W > 0 ? (W + per_split_max - 1) / per_split_max : 1;
   const int32_t max_split = W > 0 ? W : 1;
   int32_t n;
   if (request > 0) {
@@ -61,7 +72,8 @@ Plan make_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W, int32_t num_sms, 
     n = min_split;
     if (units > 0 && units < 2 * wave) {
       const int64_t want = (2 * wave + units - 1) / units;
-      const int64_t cap = W >= qsa::kMinSlotsPerSplit ? W / qsa::kMinSlotsPerSplit : 1;
+      const int64_t min_entries = (qsa::kMinSlotsPerSplit + block - 1) / block;
+      const int64_t cap = W >= min_entries ? W / min_entries : 1;
       const int64_t pick = want < cap ? want : cap;
       if (pick > n) n = int32_t(pick);
     }
@@ -116,28 +128,37 @@ const char* qsa_status_string(qsa_status_t status) {
 
 const char* qsa_last_error_detail(void) { return g_detail; }
 
-int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W,
-                                int32_t num_sms, int32_t nsplit_request,
-                                size_t* workspace_bytes) {
-  const qsa_status_t st = check_shape(Tq, Hq, Hkv, D, W);
+int32_t qsa_sparse_prefill_block_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W,
+                                      int32_t block, int32_t num_sms, int32_t nsplit_request,
+                                      size_t* workspace_bytes) {
+  qsa_status_t st = check_shape(Tq, Hq, Hkv, D, W);
+  if (st == QSA_OK) st = check_block(block);
   if (st != QSA_OK) return -int32_t(st);
   if (nsplit_request < 0) return -int32_t(fail(QSA_ERR_INVALID_ARG, "negative nsplit request"));
-  const Plan pl = make_plan(Tq, Hq, Hkv, W, num_sms, nsplit_request);
+  const Plan pl = make_plan(Tq, Hq, Hkv, W, block, num_sms, nsplit_request);
   if (workspace_bytes != nullptr) *workspace_bytes = pl.workspace;
   return pl.nsplit;
 }
 
-qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h,
-                                const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
-                                const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
-                                const int32_t* slot_idx, int64_t idx_stride_t,
-                                const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
-                                int32_t D, int64_t S, int32_t W, float scale, void* out,
-                                int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
-                                void* workspace, size_t workspace_bytes, uint32_t* err_word,
-                                void* stream) {
+int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W,
+                                int32_t num_sms, int32_t nsplit_request,
+                                size_t* workspace_bytes) {
+  return qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, 1, num_sms, nsplit_request,
+                                       workspace_bytes);
+}
+
+qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                      const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                      const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                      const int32_t* slot_idx, int64_t idx_stride_t,
+                                      const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                      int32_t D, int64_t S, int32_t W, int32_t block, float scale,
+                                      void* out, int64_t out_stride_t, int64_t out_stride_h,
+                                      int32_t nsplit, void* workspace, size_t workspace_bytes,
+                                      uint32_t* err_word, void* stream) {
   g_detail[0] = '\0';
   qsa_status_t st = check_shape(Tq, Hq, Hkv, D, W);
+  if (st == QSA_OK) st = check_block(block);
   if (st != QSA_OK) return st;
   if (S < 0) return fail(QSA_ERR_INVALID_ARG, "negative S");
   if (nsplit < 0) return fail(QSA_ERR_INVALID_ARG, "negative nsplit");
@@ -172,7 +193,7 @@ qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_str
     num_sms = device_sm_count(dev);
     if (num_sms <= 0) return fail(QSA_ERR_CUDA, "cannot query the multiprocessor count");
   }
-  const Plan pl = make_plan(Tq, Hq, Hkv, W, num_sms, nsplit);
+  const Plan pl = make_plan(Tq, Hq, Hkv, W, block, num_sms, nsplit);
   if (int64_t(Tq) * Hkv * pl.nsplit > int64_t(INT32_MAX))
     return fail(QSA_ERR_INVALID_ARG, "too many work units for one launch");
   if (pl.workspace > 0) {
@@ -215,10 +236,26 @@ qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_str
   p.k_row16 = uint32_t(k_stride_s / 8);
   p.v_row16 = uint32_t(v_stride_s / 8);
   p.scale_log2 = scale * 1.4426950408889634f;  // log2(e): the kernels use 2^x
+  p.block = block;
 
   const cudaError_t e = qsa::launch_sparse_prefill(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
   return QSA_OK;
+}
+
+qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                const int32_t* slot_idx, int64_t idx_stride_t,
+                                const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                int32_t D, int64_t S, int32_t W, float scale, void* out,
+                                int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
+                                void* workspace, size_t workspace_bytes, uint32_t* err_word,
+                                void* stream) {
+  return qsa_sparse_prefill_block(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
+                                  v_cache, v_stride_s, v_stride_h, slot_idx, idx_stride_t, width,
+                                  Tq, Hq, Hkv, D, S, W, 1, scale, out, out_stride_t, out_stride_h,
+                                  nsplit, workspace, workspace_bytes, err_word, stream);
 }
 
 }  // extern "C"

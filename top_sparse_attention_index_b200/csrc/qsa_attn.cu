@@ -108,13 +108,15 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
   const int per = (n_raw + C::kThreads - 1) / C::kThreads;
   const int b_i = min(tid * per, n_raw);
   const int e_i = min(b_i + per, n_raw);
+  // An entry is valid when its whole block of p.block slots lies in [0, S).
+  const int block = p.block;
   int cnt = 0;
   bool bad = false;
   for (int i = b_i; i < e_i; ++i) {
     const int v = sRaw[i];
-    const bool ok = v >= 0 && int64_t(v) < p.S;
+    const bool ok = v >= 0 && (int64_t(v) + 1) * block <= p.S;
     bad |= (!ok && v != -1);
-    cnt += ok ? 1 : 0;
+    cnt += ok ? block : 0;
   }
   if (bad && p.err_word != nullptr) atomicOr(p.err_word, 1u);
   int incl = cnt;
@@ -136,8 +138,12 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
     int pos = warp_off + incl - cnt;
     for (int i = b_i; i < e_i; ++i) {
       const int v = sRaw[i];
-      if (v >= 0 && int64_t(v) < p.S)
-        sOff[pos++] = make_uint2(uint32_t(v) * p.k_row16, uint32_t(v) * p.v_row16);
+      if (v >= 0 && (int64_t(v) + 1) * block <= p.S) {
+        for (int e = 0; e < block; ++e) {
+          const uint32_t slot = uint32_t(v) * uint32_t(block) + uint32_t(e);
+          sOff[pos++] = make_uint2(slot * p.k_row16, slot * p.v_row16);
+        }
+      }
     }
   }
   __syncthreads();  // sOff complete, the ring is free again

@@ -13,6 +13,7 @@ constexpr int kHeadDim = 256;           // D: the only head dimension implemente
 constexpr int kMaxGroup = 16;           // largest G = Hq / Hkv
 constexpr int kMaxSlotsPerSplit = 2560; // per-split index list staged in shared memory
 constexpr int kMinSlotsPerSplit = 128;  // the planner never makes splits narrower
+constexpr int kMaxBlock = 16;           // largest block size of block selection
 
 // Everything one launch of the fused kernel needs (passed by value).
 struct FwdParams {
@@ -37,6 +38,7 @@ struct FwdParams {
   uint32_t k_row16;         // k_stride_s / 8: one slot step of K in 16-byte units
   uint32_t v_row16;         // v_stride_s / 8
   float scale_log2;         // scale * log2(e)
+  int32_t block;            // slots named by one selected entry (1 = slot selection)
 };
 
 // Kernel configuration chosen for a group size G (shared by planner and launcher).

@@ -71,6 +71,15 @@ def work_counts(w: wl.Workload):
     return pairs, flops, gathered + other, gathered
 
 
+def reduce_max(x: float, dist=None, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -270,10 +279,7 @@ def main():
     if dist is not None:
         dist.barrier()
     kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = torch.tensor([sum(kernel_ms)], dtype=torch.float64, device=device)
-    if dist is not None:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    total_ms = float(total_ms.item())
+    total_ms = reduce_max(sum(kernel_ms), dist, device)   # the slowest rank's device time
     ms_per_step = total_ms / args.steps
 
     # end to end through the public API: pinned host inputs -> device -> kernel -> host
@@ -304,12 +310,9 @@ def main():
             e2e_step()
         ee.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([es.elapsed_time(ee) / e_steps], dtype=torch.float64, device=device)
-        if dist is not None:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": world * flops / (float(e_ms.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "ms_per_step": float(e_ms.item()), "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h}
+        e_ms = reduce_max(es.elapsed_time(ee) / e_steps, dist, device)
+        e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if dist is not None:
         dist.destroy_process_group()

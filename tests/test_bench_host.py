@@ -1,0 +1,78 @@
+"""Host-side pieces of bench.py: the work bookkeeping and the multi-rank reduction
+(world size 2 over gloo on the CPU; on GPUs the same code runs over NCCL)."""
+from __future__ import annotations
+
+import datetime
+import os
+import socket
+import sys
+from pathlib import Path
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = Path(__file__).resolve().parent.parent
+sys.path.insert(0, str(ROOT))
+
+import bench  # noqa: E402
+from top_sparse_attention_index_b200 import workloads as wl  # noqa: E402
+
+
+def test_work_counts_tiny():
+    w = wl.tiny()
+    pairs, flops, alg_bytes, gathered = bench.work_counts(w)
+    assert pairs == 124 * 64                       # four of 128 rows are fully masked
+    assert flops == pairs * 16 * 4 * 256           # 2D (QK^T) + 2D (PV) per query head
+    assert gathered == pairs * 2 * 2 * 256 * 2     # K and V rows of both KV heads, bf16
+    assert alg_bytes == gathered + 128 * 16 * 256 * 2 * 2 + 128 * 64 * 4
+
+
+def test_work_counts_width_sweep():
+    w = wl.width_sweep()
+    pairs, *_ = bench.work_counts(w)
+    ref = sum(int(((w.slot_idx[t, : int(w.width[t])] >= 0)).sum()) for t in range(w.Tq))
+    assert pairs == ref
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, queue):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    local = 10.0 + 5.0 * rank                      # rank 1 is the slow one
+    queue.put((rank, bench.reduce_max(local, dist, torch.device("cpu"))))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, queue)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(queue.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert results == {0: 15.0, 1: 15.0}
+
+
+def test_reduce_without_process_group():
+    assert bench.reduce_max(3.5) == 3.5
+
+
+def test_reference_arm_runs_on_rank0_only(capsys):
+    class A:
+        gpus, steps, warmup = 2, 1, 0
+    assert bench.run_reference(A(), rank=1) is None
+    assert capsys.readouterr().out == ""

@@ -423,3 +423,27 @@ def test_block_past_cache_end_is_flagged(cuda_device, oracle_lib):
     check_gates(out.cpu().float(), torch.from_numpy(ref), None, "block past end")
     with pytest.raises(qsa.QSAError):
         qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"], block=17)
+
+
+# ---- host-buffer API -------------------------------------------------------------------
+
+@pytest.mark.parametrize("chunk_rows", [None, 300, 7810])
+def test_sparse_prefill_from_host_matches_device_call(cuda_device, chunk_rows):
+    """The pipelined host-buffer form gives the device call's result bitwise, whatever
+    the chunking (every chunk uses the whole batch's split plan)."""
+    w = wl.long_prefill()
+    d = dev(w, cuda_device)
+    ref = qsa.sparse_prefill(d["q"], d["k_cache"], d["v_cache"], d["slot_idx"]).cpu()
+    pinned = [x.pin_memory() for x in (w.q, w.k_cache, w.v_cache, w.slot_idx)]
+    out, fin = qsa.sparse_prefill_from_host(*pinned, device=cuda_device, chunk_rows=chunk_rows)
+    fin.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
+def test_sparse_prefill_from_host_width_and_masks(cuda_device, oracle_lib):
+    w = wl.width_sweep()
+    out, fin = qsa.sparse_prefill_from_host(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width,
+                                            scale=0.05, device=cuda_device, chunk_rows=50)
+    fin.synchronize()
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 0.05)
+    check_gates(out.float(), torch.from_numpy(ref), empty_rows(w), "from_host width sweep")

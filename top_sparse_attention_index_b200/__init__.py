@@ -27,10 +27,11 @@ from ._binding import (  # noqa: F401
     qsa_sparse_prefill_plan,
     qsa_status_string,
     sparse_prefill,
+    sparse_prefill_from_host,
 )
 
 __all__ = [
-    "sparse_prefill", "qsa_sparse_prefill", "qsa_sparse_prefill_noalloc",
+    "sparse_prefill", "sparse_prefill_from_host", "qsa_sparse_prefill", "qsa_sparse_prefill_noalloc",
     "qsa_sparse_prefill_block", "qsa_sparse_prefill_block_plan",
     "qsa_sparse_prefill_plan", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
     "load_library", "QSAError",

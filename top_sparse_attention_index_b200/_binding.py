@@ -207,3 +207,84 @@ def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=No
     if st != QSA_OK:
         raise QSAError(st, qsa_last_error_detail())
     return out
+
+
+_COPY_STREAMS = {}
+
+
+def _copy_streams(device):
+    """The two side streams of the host-buffer path, one pair per device, created once:
+    reusing them lets the caching allocator recycle the staging buffers of earlier
+    calls instead of allocating (and synchronising) anew."""
+    key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    if key not in _COPY_STREAMS:
+        _COPY_STREAMS[key] = (torch.cuda.Stream(key), torch.cuda.Stream(key))
+    return _COPY_STREAMS[key]
+
+
+def sparse_prefill_from_host(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=None,
+                             device=None, chunk_rows=None, nsplit=0, block=1):
+    """Host-buffer form of sparse_prefill: copies the inputs to `device`, runs the kernels
+    and copies the result back, overlapping the transfers with the computation.
+
+    Inputs are CPU tensors (pinned memory makes the copies asynchronous); the result is
+    written to `out` (a CPU bf16 [Tq, Hq, 256] tensor, allocated pinned when None) and
+    is complete when the returned CUDA event has completed (``event.synchronize()``).
+    K and V are copied first (every query row may read any slot); then query rows go in
+    chunks of `chunk_rows`: chunk c+1's Q and indices cross the bus while chunk c is
+    computed and chunk c-1's output returns on a third stream.  With nsplit = 0 every
+    chunk uses the split plan of the whole batch, so the result is bitwise that of
+    sparse_prefill on the whole batch whatever the chunking.
+    """
+    device = torch.device(device if device is not None else "cuda")
+    if device.type != "cuda":
+        raise ValueError("sparse_prefill_from_host needs a CUDA device")
+    Tq, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(Tq, Hq, D, dtype=torch.bfloat16).pin_memory()
+    if chunk_rows is None:
+        chunk_rows = max(-(-Tq // 16), 256)
+    if nsplit == 0:
+        # every chunk uses the whole batch's split plan, so the result does not depend
+        # on the chunking: it is bitwise that of one device call on the whole batch
+        num_sms = torch.cuda.get_device_properties(device).multi_processor_count
+        nsplit, _ = qsa_sparse_prefill_block_plan(Tq, Hq, k_cache.shape[1], D, slot_idx.shape[1],
+                                                  block, num_sms, 0)
+    h2d, d2h = _copy_streams(device)
+    comp = torch.cuda.current_stream(device)
+    h2d.wait_stream(comp)  # ordered after work already queued on the caller's stream
+    with torch.cuda.device(device):
+        with torch.cuda.stream(h2d):
+            k_d = k_cache.to(device, non_blocking=True)
+            v_d = v_cache.to(device, non_blocking=True)
+            kv_ready = torch.cuda.Event()
+            kv_ready.record(h2d)
+        out_d = torch.empty(Tq, Hq, D, dtype=torch.bfloat16, device=device)
+        comp.wait_event(kv_ready)
+        done = None
+        for r0 in range(0, max(Tq, 1), chunk_rows):
+            r1 = min(Tq, r0 + chunk_rows)
+            with torch.cuda.stream(h2d):
+                q_c = q[r0:r1].to(device, non_blocking=True)
+                i_c = slot_idx[r0:r1].to(device, non_blocking=True)
+                w_c = None if width is None else width[r0:r1].to(device, non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(h2d)
+            comp.wait_event(ready)
+            # the chunk's device buffers were allocated on h2d and are used on comp
+            for t in (q_c, i_c, w_c):
+                if t is not None:
+                    t.record_stream(comp)
+            sparse_prefill(q_c, k_d, v_d, i_c, w_c, scale=scale, out=out_d[r0:r1], nsplit=nsplit,
+                           stream=comp, block=block)
+            done = torch.cuda.Event()
+            done.record(comp)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                out[r0:r1].copy_(out_d[r0:r1], non_blocking=True)
+        for t in (k_d, v_d):
+            t.record_stream(comp)
+        out_d.record_stream(d2h)
+        finished = torch.cuda.Event()
+        finished.record(d2h)
+    return out, finished

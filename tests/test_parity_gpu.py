@@ -447,3 +447,44 @@ def test_sparse_prefill_from_host_width_and_masks(cuda_device, oracle_lib):
     fin.synchronize()
     ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 0.05)
     check_gates(out.float(), torch.from_numpy(ref), empty_rows(w), "from_host width sweep")
+
+
+# ---- maximum sizes ----------------------------------------------------------------------
+
+def test_large_cache_two_million_slots(cuda_device, oracle_lib):
+    """S = 2,097,152 slots at Hkv = 2 (2 GiB each for K and V on the device).  Only the
+    selected rows hold data; the oracle runs on a compact copy of those rows with the
+    indices renumbered (the definition does not depend on where a row lives)."""
+    S, Hq, Hkv, Tq, W = 1 << 21, 16, 2, 64, 2051
+    g = torch.Generator().manual_seed(401)
+    idx = wl.uniform_distinct(g, Tq, S, W)
+    idx[:, ::7] = -1
+    used = torch.unique(idx[idx >= 0])
+    rows_k = torch.randn(used.numel(), Hkv, D, generator=g).to(torch.bfloat16)
+    rows_v = torch.randn(used.numel(), Hkv, D, generator=g).to(torch.bfloat16)
+    q = torch.randn(Tq, Hq, D, generator=g).to(torch.bfloat16)
+    k_dev = torch.zeros(S, Hkv, D, dtype=torch.bfloat16, device=cuda_device)
+    v_dev = torch.zeros(S, Hkv, D, dtype=torch.bfloat16, device=cuda_device)
+    k_dev[used.to(cuda_device)] = rows_k.to(cuda_device)
+    v_dev[used.to(cuda_device)] = rows_v.to(cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = qsa.sparse_prefill(q.to(cuda_device), k_dev, v_dev, idx.to(cuda_device), err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    remap = torch.full((S,), -1, dtype=torch.int32)
+    remap[used] = torch.arange(used.numel(), dtype=torch.int32)
+    idx_c = torch.where(idx >= 0, remap[idx.clamp(min=0).long()], idx)
+    ref = oracle_lib.forward(q, rows_k, rows_v, idx_c, None, 1.0 / 16.0)
+    check_gates(out.cpu().float(), torch.from_numpy(ref), None, "2M-slot cache")
+    del k_dev, v_dev
+
+
+def test_very_wide_selection(cuda_device, oracle_lib):
+    """W = 20,000 selected slots per row: at least eight splits, combined by the LSE
+    kernel."""
+    w = _random_case(402, 40, 16, 2, 65536, 20000, minus1=0.05, widths=True)
+    n, _ = qsa.qsa_sparse_prefill_plan(40, 16, 2, D, 20000, 148)
+    assert n >= 8
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    rows = list(range(0, 40, 3))
+    compare_rows(w, got, oracle_lib, 1.0 / 16.0, rows, "W=20000")

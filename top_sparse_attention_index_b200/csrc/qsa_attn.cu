@@ -243,11 +243,22 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
 #pragma unroll
   for (int mt = 0; mt < 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
-  const int key = lane & 7;  // swizzle key of every row this lane addresses
+  // ldmatrix addressing.  Chunk c of a row sits at ((c ^ key) << 4), key = row & 7 =
+  // lane & 7 for every row this lane addresses.  With c = 2 * step + hi (step = k-step
+  // for K, m-tile for V; hi in {0, 1}) the XOR only touches the low three bits, so
+  // (c ^ key) << 4 = 128 * (step >> 2) + swz[step & 3]: four per-lane offsets computed
+  // once, and every ldmatrix address in the loop is a register plus an immediate.
+  const int key = lane & 7;
   const int krow = (lane & 7) + ((lane >> 3) & 1) * 8;
   const int khi = lane >> 4;
   const int vrow = (lane & 7) + ((lane >> 4) << 3);
   const int vhi = (lane >> 3) & 1;
+  uint32_t kswz[4], vswz[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    kswz[m] = uint32_t(krow * kRowBytes + (((2 * m + khi) ^ key) << 4));
+    vswz[m] = uint32_t(16 * kRowBytes + vrow * kRowBytes + (((2 * m + vhi) ^ key) << 4));
+  }
   const float sl2 = p.scale_log2;
 
   for (int s = 0; s < n_stages; ++s) {
@@ -264,14 +275,16 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
     const uint32_t sub = sub_s + buf * C::kSubBytes;
 
     // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8); two chains for ILP.
-    const uint32_t kt = sub + krow * kRowBytes;
+    uint32_t kt[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) kt[m] = sub + kswz[m];
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 16; ks += 2) {
       uint32_t a[4];
-      ldmatrix_x4(a, kt + (((2 * ks + khi) ^ key) << 4));
+      ldmatrix_x4(a, kt[ks & 3] + 128 * (ks >> 2));
       mma_bf16_16816(sa, a, qf[ks][0], qf[ks][1]);
-      ldmatrix_x4(a, kt + (((2 * ks + 2 + khi) ^ key) << 4));
+      ldmatrix_x4(a, kt[(ks + 1) & 3] + 128 * ((ks + 1) >> 2));
       mma_bf16_16816(sb, a, qf[ks + 1][0], qf[ks + 1][1]);
     }
     float x0 = (sa[0] + sb[0]) * sl2, x1 = (sa[1] + sb[1]) * sl2;
@@ -316,11 +329,13 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
     // O^T (256 x 8) += V^T (256 x 16) * P^T (16 x 8)
     const uint32_t b0 = movmatrix_trans(p01);
     const uint32_t b1 = movmatrix_trans(p23);
-    const uint32_t vt = sub + 16 * kRowBytes + vrow * kRowBytes;
+    uint32_t vt[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m];
 #pragma unroll
     for (int mt = 0; mt < 16; ++mt) {
       uint32_t a[4];
-      ldmatrix_x4_trans(a, vt + (((2 * mt + vhi) ^ key) << 4));
+      ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
       mma_bf16_16816(o[mt], a, b0, b1);
     }
   }

@@ -35,6 +35,18 @@ sys.path.insert(0, str(ROOT))
 from top_sparse_attention_index_b200 import workloads as wl  # noqa: E402
 
 METRIC = "sparse prefill TFLOP/s & query-slot pairs/s, 7810q×2051 sel; % of roofline"
+
+# The five configurations (see workloads.py); the benchmark line is long_prefill.
+WORKLOADS = {
+    "long_prefill": lambda: wl.long_prefill(),
+    "tiny": lambda: wl.tiny(),
+    "width_sweep": lambda: wl.width_sweep(),
+    "causal_two_request": lambda: wl.causal_two_request(),
+    "max_extent_g6_uniform": lambda: wl.max_extent(6, False),
+    "max_extent_g6_clustered": lambda: wl.max_extent(6, True),
+    "max_extent_g3_uniform": lambda: wl.max_extent(3, False),
+    "max_extent_g3_clustered": lambda: wl.max_extent(3, True),
+}
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 512 << 20
 
@@ -52,18 +64,25 @@ def parse_args():
     ap.add_argument("--rows", type=int, default=0,
                     help="keep only the first ROWS query rows (small cases for ncu captures, "
                          "decode-like batches)")
+    ap.add_argument("--workload", default="long_prefill", choices=sorted(WORKLOADS),
+                    help="workload to time (the default is the benchmark's)")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of a CUDA graph that holds one step")
     return ap.parse_args()
 
 
+def pairs_per_row(w: wl.Workload) -> torch.Tensor:
+    """Valid (t, slot) pairs of every query row (int64 [Tq])."""
+    pos = torch.arange(w.W)[None, :]
+    wt = torch.full((w.Tq, 1), w.W) if w.width is None else w.width.to(torch.int64)[:, None]
+    ok = (pos < wt) & (w.slot_idx >= 0) & (w.slot_idx < w.S)
+    return ok.sum(dim=1)
+
+
 def work_counts(w: wl.Workload):
     """Valid (t, slot) pairs and the algorithmic FLOPs / bytes of one pass."""
     W = w.W
-    pos = torch.arange(W)[None, :]
-    wt = torch.full((w.Tq, 1), W) if w.width is None else w.width.to(torch.int64)[:, None]
-    ok = (pos < wt) & (w.slot_idx >= 0) & (w.slot_idx < w.S)
-    pairs = int(ok.sum())
+    pairs = int(pairs_per_row(w).sum())
     D = w.q.shape[2]
     flops = pairs * w.Hq * 4 * D                         # 2D (QK^T) + 2D (PV) per head
     gathered = pairs * w.Hkv * 2 * D * 2                 # K and V rows, bf16
@@ -152,20 +171,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_baseline(w: wl.Workload, flops_per_row: float, target_s: float):
+def cpu_baseline(w: wl.Workload, target_s: float):
     """The oracle as it stands on the host cores, on a bounded sample of query rows."""
     import oracle
     o = oracle.default()
-    probe = list(range(16))
+    scale = w.scales[0]
+    probe = list(range(min(16, w.Tq)))
     t0 = time.perf_counter()
-    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0, rows=probe)
+    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=probe)
     dt = max(time.perf_counter() - t0, 1e-3)
     n = int(min(w.Tq, max(64, len(probe) * target_s / dt)))
     rows = list(range(n))
     t0 = time.perf_counter()
-    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0, rows=rows)
+    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=rows)
     dt = time.perf_counter() - t0
-    flops = flops_per_row * n  # every row of this workload has the same valid width
+    flops = int(pairs_per_row(w)[:n].sum()) * w.Hq * 4 * 256
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": o.num_threads(),
             "kind": "oracle", "seconds": round(dt, 3),
             "sample": f"first {n} of {w.Tq} query rows of the same workload (all heads, all selected slots)"}
@@ -229,12 +249,15 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
 
-    w = wl.long_prefill()
+    w = WORKLOADS[args.workload]()
     if args.rows:
         w = wl.Workload(f"{w.name}_rows{args.rows}", w.q[:args.rows], w.k_cache, w.v_cache,
-                        w.slot_idx[:args.rows], None)
+                        w.slot_idx[:args.rows], None if w.width is None else w.width[:args.rows],
+                        scales=w.scales)
     pairs, flops, alg_bytes, gathered = work_counts(w)
     q, k, v, idx = (x.to(device) for x in (w.q, w.k_cache, w.v_cache, w.slot_idx))
+    width = None if w.width is None else w.width.to(device)
+    scale = w.scales[0]
     out = torch.empty(w.Tq, w.Hq, 256, dtype=torch.bfloat16, device=device)
     num_sms = torch.cuda.get_device_properties(device).multi_processor_count
     nsplit, ws_bytes = qsa.qsa_sparse_prefill_plan(w.Tq, w.Hq, w.Hkv, 256, w.W, num_sms)
@@ -243,7 +266,7 @@ def main():
     stream = torch.cuda.current_stream(device)
 
     def step():
-        qsa.sparse_prefill(q, k, v, idx, scale=1.0 / 16.0, out=out)
+        qsa.sparse_prefill(q, k, v, idx, width, scale=scale, out=out)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -292,8 +315,8 @@ def main():
         d2h = hout.numel() * hout.element_size()
 
         def e2e_step():
-            _, fin = qsa.sparse_prefill_from_host(hq, hk, hv, hidx, scale=1.0 / 16.0, out=hout,
-                                                  device=device)
+            _, fin = qsa.sparse_prefill_from_host(hq, hk, hv, hidx, w.width, scale=scale,
+                                                  out=hout, device=device)
             return fin
 
         for _ in range(3):
@@ -354,7 +377,7 @@ def main():
     if e2e is not None:
         result["e2e"] = e2e
     if not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, flops / w.Tq, args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(result))
 
 

@@ -107,4 +107,6 @@ def check_gates(got: torch.Tensor, ref: torch.Tensor, empty_rows=None, label="")
     if empty_rows is not None and len(empty_rows):
         z = got[list(empty_rows)]
         assert (z == 0).all(), f"{label}: empty rows are not exactly zero"
-    return err.max().item() if err.numel() else 0.0, rel
+    max_err = err.max().item() if err.numel() else 0.0
+    print(f"PARITY {label}: rows={got.shape[0]} max_abs_err={max_err:.3e} rel_l2={rel:.3e}")
+    return max_err, rel

@@ -39,6 +39,7 @@ METRIC = "sparse prefill TFLOP/s & query-slot pairs/s, 7810q×2051 sel; % of roo
 # The five configurations (see workloads.py); the benchmark line is long_prefill.
 WORKLOADS = {
     "long_prefill": lambda: wl.long_prefill(),
+    "long_prefill_block4": lambda: wl.long_prefill_block4(),
     "tiny": lambda: wl.tiny(),
     "width_sweep": lambda: wl.width_sweep(),
     "causal_two_request": lambda: wl.causal_two_request(),
@@ -72,11 +73,12 @@ def parse_args():
 
 
 def pairs_per_row(w: wl.Workload) -> torch.Tensor:
-    """Valid (t, slot) pairs of every query row (int64 [Tq])."""
+    """Valid (t, slot) pairs of every query row (int64 [Tq]); with block selection every
+    valid entry names w.block slots."""
     pos = torch.arange(w.W)[None, :]
     wt = torch.full((w.Tq, 1), w.W) if w.width is None else w.width.to(torch.int64)[:, None]
-    ok = (pos < wt) & (w.slot_idx >= 0) & (w.slot_idx < w.S)
-    return ok.sum(dim=1)
+    ok = (pos < wt) & (w.slot_idx >= 0) & ((w.slot_idx.to(torch.int64) + 1) * w.block <= w.S)
+    return ok.sum(dim=1) * w.block
 
 
 def work_counts(w: wl.Workload):
@@ -85,7 +87,7 @@ def work_counts(w: wl.Workload):
     pairs = int(pairs_per_row(w).sum())
     D = w.q.shape[2]
     flops = pairs * w.Hq * 4 * D                         # 2D (QK^T) + 2D (PV) per head
-    gathered = pairs * w.Hkv * 2 * D * 2                 # K and V rows, bf16
+    gathered = pairs * w.Hkv * 2 * D * 2                 # K and V rows, bf16 (pairs count slots)
     other = w.Tq * w.Hq * D * 2 * 2 + w.Tq * W * 4       # Q in, out, indices
     return pairs, flops, gathered + other, gathered
 
@@ -178,12 +180,12 @@ def cpu_baseline(w: wl.Workload, target_s: float):
     scale = w.scales[0]
     probe = list(range(min(16, w.Tq)))
     t0 = time.perf_counter()
-    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=probe)
+    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=probe, block=w.block)
     dt = max(time.perf_counter() - t0, 1e-3)
     n = int(min(w.Tq, max(64, len(probe) * target_s / dt)))
     rows = list(range(n))
     t0 = time.perf_counter()
-    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=rows)
+    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=rows, block=w.block)
     dt = time.perf_counter() - t0
     flops = int(pairs_per_row(w)[:n].sum()) * w.Hq * 4 * 256
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": o.num_threads(),
@@ -253,20 +255,21 @@ def main():
     if args.rows:
         w = wl.Workload(f"{w.name}_rows{args.rows}", w.q[:args.rows], w.k_cache, w.v_cache,
                         w.slot_idx[:args.rows], None if w.width is None else w.width[:args.rows],
-                        scales=w.scales)
+                        scales=w.scales, block=w.block)
     pairs, flops, alg_bytes, gathered = work_counts(w)
     q, k, v, idx = (x.to(device) for x in (w.q, w.k_cache, w.v_cache, w.slot_idx))
     width = None if w.width is None else w.width.to(device)
     scale = w.scales[0]
     out = torch.empty(w.Tq, w.Hq, 256, dtype=torch.bfloat16, device=device)
     num_sms = torch.cuda.get_device_properties(device).multi_processor_count
-    nsplit, ws_bytes = qsa.qsa_sparse_prefill_plan(w.Tq, w.Hq, w.Hkv, 256, w.W, num_sms)
+    nsplit, ws_bytes = qsa.qsa_sparse_prefill_block_plan(w.Tq, w.Hq, w.Hkv, 256, w.W, w.block,
+                                                         num_sms)
     launches_per_step = 1 if nsplit == 1 else 2
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step():
-        qsa.sparse_prefill(q, k, v, idx, width, scale=scale, out=out)
+        qsa.sparse_prefill(q, k, v, idx, width, scale=scale, out=out, block=w.block)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -316,7 +319,7 @@ def main():
 
         def e2e_step():
             _, fin = qsa.sparse_prefill_from_host(hq, hk, hv, hidx, w.width, scale=scale,
-                                                  out=hout, device=device)
+                                                  out=hout, device=device, block=w.block)
             return fin
 
         for _ in range(3):
@@ -344,7 +347,7 @@ def main():
     prof = ROOT / "profiles" / "traffic.json"
     if prof.exists():
         tj = json.loads(prof.read_text())
-        if tj.get("kernel_source_hash") == _kernel_hash():
+        if tj.get("kernel_source_hash") == _kernel_hash() and tj.get("workload_name") == w.name:
             traffic = tj.get("bytes_per_launch")
     result = {
         "metric": METRIC,
@@ -382,10 +385,12 @@ def main():
 
 
 def _kernel_hash():
+    """Hash of the kernel sources (the DRAM traffic record is valid while it matches)."""
     import hashlib
     h = hashlib.sha256()
-    for p in sorted((ROOT / "top_sparse_attention_index_b200" / "csrc").glob("*")):
-        h.update(p.read_bytes())
+    csrc = ROOT / "top_sparse_attention_index_b200" / "csrc"
+    for name in ("qsa_attn.cu", "qsa_internal.h", "qsa_ptx.cuh"):
+        h.update((csrc / name).read_bytes())
     return h.hexdigest()[:16]
 
 

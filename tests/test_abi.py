@@ -65,9 +65,13 @@ def test_plan_without_split(lib, Tq, Hq, Hkv, W, expect):
 
 
 def test_plan_splits_small_batches(lib):
-    n, ws = qsa.qsa_sparse_prefill_plan(257, 12, 1, 256, 2051, 148)
-    assert n > 1
-    assert ws >= n * 257 * 12 * 256 * 4 + n * 257 * 12 * 4
+    # 16 rows x 2 KV heads = 32 units: floor(148 / 32) = 4 splits fill one wave
+    n, ws = qsa.qsa_sparse_prefill_plan(16, 16, 2, 256, 2051, 148)
+    assert n == 4
+    assert ws >= n * 16 * 16 * 256 * 4 + n * 16 * 16 * 4
+    # one wave or more of units: no split
+    assert qsa.qsa_sparse_prefill_plan(64, 16, 2, 256, 2051, 148)[0] == 1
+    assert qsa.qsa_sparse_prefill_plan(257, 12, 1, 256, 2051, 148)[0] == 1
     n1, _ = qsa.qsa_sparse_prefill_plan(1, 16, 2, 256, 2051, 148)
     assert n1 == 16  # floor(2051 / 128): splits are never narrower than 128 positions
     assert -(-2051 // n1) >= 128

@@ -334,7 +334,7 @@ def _raw_call(d, out, ws, nsplit, stream):
         stream)
 
 
-@pytest.mark.parametrize("Tq", [1, 8, 64])
+@pytest.mark.parametrize("Tq", [1, 8, 16, 64])
 def test_cuda_graph_capture_decode_shape(cuda_device, oracle_lib, Tq):
     """Few query rows with a wide selection (all parallelism from split-W plus the
     combine kernel).  The call only enqueues kernels on the given stream, so it can be
@@ -345,8 +345,9 @@ def test_cuda_graph_capture_decode_shape(cuda_device, oracle_lib, Tq):
     d = dev(cases[0], cuda_device)
     num_sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
     nsplit, ws_bytes = qsa.qsa_sparse_prefill_plan(Tq, 16, 2, D, 2051, num_sms)
-    assert nsplit > 1
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=cuda_device)
+    if Tq * 2 < num_sms // 2:
+        assert nsplit > 1
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=cuda_device)
     out = torch.empty(Tq, 16, D, dtype=torch.bfloat16, device=cuda_device)
     # one eager call first: it sets the kernels' per-device attributes
     assert _raw_call(d, out, ws, nsplit, torch.cuda.current_stream().cuda_stream) == qsa.QSA_OK

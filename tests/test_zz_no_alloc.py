@@ -23,7 +23,7 @@ pytestmark = pytest.mark.gpu
 D = 256
 
 
-def _case(seed, Tq=64, Hq=16, Hkv=2, S=65536, W=2051):
+def _case(seed, Tq=16, Hq=16, Hkv=2, S=65536, W=2051):
     g = torch.Generator().manual_seed(seed)
     q = torch.randn(Tq, Hq, D, generator=g).to(torch.bfloat16)
     k = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)

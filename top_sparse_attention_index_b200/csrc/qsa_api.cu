@@ -53,8 +53,8 @@ qsa_status_t check_shape(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t
 }
 
 // Splits of the W axis.  One split's slots (entries x block) must fit the shared-memory
-// offset list; with few work units, more splits fill about two waves of CTAs but none
-// is narrower than kMinSlotsPerSplit slots.
+// offset list; with fewer work units than one wave of CTAs, more splits fill that wave
+// but none is narrower than kMinSlotsPerSplit slots.
 Plan make_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W, int32_t block, int32_t num_sms,
                int32_t request) {
   const int32_t G = Hq / Hkv;
@@ -65,13 +65,15 @@ Plan make_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W, int32_t block, in
   if (request > 0) {
     n = request < min_split ? min_split : (request > max_split ? max_split : request);
   } else {
-    // Enough CTAs for about two waves; never splits narrower than kMinSlotsPerSplit.
+    // Fewer work units than one wave of CTAs: split W until the CTAs fill (at most) one
+    // wave -- more splits cost more than the extra parallelism gives (measured on
+    // decode-shape batches); never splits narrower than kMinSlotsPerSplit.
     const qsa::KernelShape ks = qsa::kernel_shape(G);
     const int64_t wave = int64_t(num_sms > 0 ? num_sms : 1) * ks.ctas_per_sm;
     const int64_t units = int64_t(Tq) * Hkv;
     n = min_split;
-    if (units > 0 && units < 2 * wave) {
-      const int64_t want = (2 * wave + units - 1) / units;
+    if (units > 0 && units < wave) {
+      const int64_t want = wave / units;
       const int64_t min_entries = (qsa::kMinSlotsPerSplit + block - 1) / block;
       const int64_t cap = W >= min_entries ? W / min_entries : 1;
       const int64_t pick = want < cap ? want : cap;

@@ -40,6 +40,7 @@ class Workload:
     width: torch.Tensor | None  # int32 [Tq] or None (= W)
     scales: tuple = (DEFAULT_SCALE,)
     notes: dict = field(default_factory=dict)
+    block: int = 1              # slots named by one entry of slot_idx (block selection)
 
     @property
     def Tq(self) -> int:
@@ -204,6 +205,19 @@ def long_prefill(seed: int = 1238) -> Workload:
     q, k, v = _qkv(gen, Tq, Hq, Hkv, S)
     idx = uniform_distinct(gen, Tq, S, W)
     return Workload("long_prefill_hq16_hkv2_s65536_tq7810_w2051", q, k, v, idx, None)
+
+
+def long_prefill_block4(seed: int = 1244) -> Workload:
+    """Block selection at the indexer's budget ("Why QSA is the awkward part, in
+    numbers": 2,048 selected micro-blocks per query, compression ratio 4): Hq=16, Hkv=2,
+    S=65,536, Tq=7,810, W=2,048 distinct blocks of 4 consecutive slots per row (8,192
+    slots), uniform over the 16,384 blocks of the cache."""
+    gen = torch.Generator().manual_seed(seed)
+    Tq, Hq, Hkv, S, W, B = 7810, 16, 2, 65536, 2048, 4
+    q, k, v = _qkv(gen, Tq, Hq, Hkv, S)
+    idx = uniform_distinct(gen, Tq, S // B, W)
+    return Workload("long_prefill_block4_hq16_hkv2_s65536_tq7810_w2048x4", q, k, v, idx, None,
+                    block=B)
 
 
 def max_extent(Hq: int = 6, clustered: bool = False, seed: int | None = None) -> Workload:

@@ -180,28 +180,37 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
   // Pad the offset list to whole 16-slot sub-tiles with the first slot: padding rows
   // hold finite data and are masked out of the softmax.
   for (int i = n_valid + tid; i < ((n_valid + 15) & ~15); i += C::kThreads) sOff[i] = sOff[0];
-  const char* kbase = reinterpret_cast<const char*>(p.k_cache + int64_t(j) * p.k_stride_h) + lane * 16;
-  const char* vbase = reinterpret_cast<const char*>(p.v_cache + int64_t(j) * p.v_stride_h) + lane * 16;
+  // Gather addressing: global-space row bases (one mad.wide per row and tensor in the
+  // loop) and, per lane, the eight swizzled chunk offsets (row & 7 is a compile-time
+  // constant in the unrolled loop because a lane's rows start at 0 or 8), so a
+  // destination is a register plus an immediate.
+  const uint64_t kg = static_cast<uint64_t>(__cvta_generic_to_global(
+                          p.k_cache + int64_t(j) * p.k_stride_h)) + uint64_t(lane) * 16;
+  const uint64_t vg = static_cast<uint64_t>(__cvta_generic_to_global(
+                          p.v_cache + int64_t(j) * p.v_stride_h)) + uint64_t(lane) * 16;
   const uint32_t lane16 = uint32_t(lane) << 4;
   // this lane's sub-tiles: [wslot][stage]; a warp pair splits the 16 rows 8 / 8
   const uint32_t sub_s = ring_s + wslot * STAGES * C::kSubBytes;
   constexpr int kLoadRows = 16 / NTILE;
   const int row0 = wn * kLoadRows;
+  const uint32_t sub_rows = sub_s + row0 * kRowBytes;
 
   auto load_stage = [&](int s, int buf) {
     const int base = s * C::kRows + wslot * 16;
     if (base >= n_valid) return;  // an empty sub-tile is neither loaded nor read
-    const uint32_t kdst = sub_s + buf * C::kSubBytes;
+    uint32_t kd[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (m << 4));
+    const uint4* offs = reinterpret_cast<const uint4*>(sOff + base + row0);  // 16-byte aligned
 #pragma unroll
     for (int i = 0; i < kLoadRows; i += 2) {
-      const uint4 o2 = *reinterpret_cast<const uint4*>(sOff + base + row0 + i);  // rows r, r+1
-      const int r = row0 + i;
-      const uint32_t d0 = kdst + r * kRowBytes + (lane16 ^ ((r & 7) << 4));
-      const uint32_t d1 = kdst + (r + 1) * kRowBytes + (lane16 ^ (((r + 1) & 7) << 4));
-      cp_async_16(d0, kbase + size_t(o2.x) * 16);
-      cp_async_16(d0 + 16 * kRowBytes, vbase + size_t(o2.y) * 16);
-      cp_async_16(d1, kbase + size_t(o2.z) * 16);
-      cp_async_16(d1 + 16 * kRowBytes, vbase + size_t(o2.w) * 16);
+      const uint4 o2 = offs[i / 2];  // offsets of rows i and i + 1
+      const uint32_t d0 = kd[i & 7] + i * kRowBytes;
+      const uint32_t d1 = kd[(i + 1) & 7] + (i + 1) * kRowBytes;
+      cp_async_16_global(d0, kg + uint64_t(o2.x) * 16);
+      cp_async_16_global(d0 + 16 * kRowBytes, vg + uint64_t(o2.y) * 16);
+      cp_async_16_global(d1, kg + uint64_t(o2.z) * 16);
+      cp_async_16_global(d1 + 16 * kRowBytes, vg + uint64_t(o2.w) * 16);
     }
   };
   // makes a stage's sub-tile, loaded by one warp or a warp pair, visible to it

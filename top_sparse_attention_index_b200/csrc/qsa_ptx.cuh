@@ -28,6 +28,11 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
 }
 
+// 16-byte async copy from a global-space address (from __cvta_generic_to_global).
+__device__ __forceinline__ void cp_async_16_global(uint32_t dst, uint64_t gaddr) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(gaddr) : "memory");
+}
+
 // Barrier `id` (1..15) over `threads` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");

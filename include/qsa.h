@@ -66,7 +66,7 @@ typedef enum {
 
 /* Largest number of selected positions one split processes (the per-split index list
  * is staged whole in shared memory).  Wider selections are split automatically. */
-#define QSA_MAX_SLOTS_PER_SPLIT 2560
+#define QSA_MAX_SLOTS_PER_SPLIT 2240
 
 /* Version of this ABI; bumped on any signature change. */
 int32_t qsa_abi_version(void);

@@ -65,20 +65,21 @@ def test_plan_without_split(lib, Tq, Hq, Hkv, W, expect):
 
 
 def test_plan_splits_small_batches(lib):
-    # 16 rows x 2 KV heads = 32 units: floor(148 / 32) = 4 splits fill one wave
+    # 16 rows x 2 KV heads = 32 units; one wave = 148 SMs x 2 resident CTAs = 296:
+    # floor(296 / 32) = 9 splits fill it
     n, ws = qsa.qsa_sparse_prefill_plan(16, 16, 2, 256, 2051, 148)
-    assert n == 4
+    assert n == 9
     assert ws >= n * 16 * 16 * 256 * 4 + n * 16 * 16 * 4
     # one wave or more of units: no split
-    assert qsa.qsa_sparse_prefill_plan(64, 16, 2, 256, 2051, 148)[0] == 1
-    assert qsa.qsa_sparse_prefill_plan(257, 12, 1, 256, 2051, 148)[0] == 1
+    assert qsa.qsa_sparse_prefill_plan(160, 16, 2, 256, 2051, 148)[0] == 1
+    assert qsa.qsa_sparse_prefill_plan(300, 12, 1, 256, 2051, 148)[0] == 1
     n1, _ = qsa.qsa_sparse_prefill_plan(1, 16, 2, 256, 2051, 148)
     assert n1 == 16  # floor(2051 / 128): splits are never narrower than 128 positions
     assert -(-2051 // n1) >= 128
 
 
 def test_block_plan(lib):
-    # 2,048 blocks of 4 = 8,192 slots per row: at least ceil(8192 / 2560) = 4 splits
+    # 2,048 blocks of 4 = 8,192 slots per row: ceil(8192 / 2240) = 4 splits
     n, ws = qsa.qsa_sparse_prefill_block_plan(7810, 16, 2, 256, 2048, 4, 148)
     assert n == 4 and ws > 0
     assert qsa.qsa_sparse_prefill_block_plan(7810, 16, 2, 256, 2051, 1, 148) == \
@@ -91,7 +92,7 @@ def test_block_plan(lib):
 
 def test_plan_wide_rows_force_splits(lib):
     n, _ = qsa.qsa_sparse_prefill_plan(100000, 16, 2, 256, 6000, 148)
-    assert n == 3  # ceil(6000 / 2560)
+    assert n == 3  # ceil(6000 / 2240)
     n, _ = qsa.qsa_sparse_prefill_plan(100000, 16, 2, 256, 6000, 148, 1)
     assert n == 3  # a request below the minimum is raised
     n, _ = qsa.qsa_sparse_prefill_plan(10, 16, 2, 256, 5, 148, 64)
@@ -147,7 +148,7 @@ INVALID = [
     (dict(scale=float("nan")), qsa.QSA_ERR_INVALID_ARG),
     (dict(scale=float("inf")), qsa.QSA_ERR_INVALID_ARG),
     (dict(nsplit=-2), qsa.QSA_ERR_INVALID_ARG),
-    (dict(S=2 ** 30), qsa.QSA_ERR_UNSUPPORTED),           # K rows beyond 64 GiB reach
+    (dict(k_stride_s=2 ** 31), qsa.QSA_ERR_UNSUPPORTED),  # slot stride of 4 GiB
     (dict(nsplit=2, W=8, workspace=None), qsa.QSA_ERR_WORKSPACE),
     (dict(nsplit=2, W=8, workspace=0x70000, workspace_bytes=16), qsa.QSA_ERR_WORKSPACE),
 ]

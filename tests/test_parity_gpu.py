@@ -174,7 +174,7 @@ def test_forced_splits_decode_shape(cuda_device, oracle_lib, nsplit):
 
 
 def test_rows_wider_than_one_split(cuda_device, oracle_lib):
-    """W = 6,000 > 2,560 positions per split forces at least three splits."""
+    """W = 6,000 > 2,240 slots per split forces at least three splits."""
     w = _random_case(78, 300, 16, 2, 20000, 6000, minus1=0.1, widths=True)
     n, _ = qsa.qsa_sparse_prefill_plan(w.Tq, 16, 2, D, w.W, 148)
     assert n >= 3
@@ -345,7 +345,7 @@ def test_cuda_graph_capture_decode_shape(cuda_device, oracle_lib, Tq):
     d = dev(cases[0], cuda_device)
     num_sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
     nsplit, ws_bytes = qsa.qsa_sparse_prefill_plan(Tq, 16, 2, D, 2051, num_sms)
-    if Tq * 2 < num_sms // 2:
+    if Tq * 2 < num_sms:
         assert nsplit > 1
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=cuda_device)
     out = torch.empty(Tq, 16, D, dtype=torch.bfloat16, device=cuda_device)

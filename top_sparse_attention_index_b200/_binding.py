@@ -21,7 +21,7 @@ QSA_ERR_WORKSPACE = 3
 QSA_ERR_CUDA = 4
 QSA_ERRBIT_SLOT_RANGE = 0x1
 QSA_ERRBIT_WIDTH_RANGE = 0x2
-QSA_MAX_SLOTS_PER_SPLIT = 2560
+QSA_MAX_SLOTS_PER_SPLIT = 2240
 QSA_MAX_BLOCK = 16
 QSA_STATIC_SCRATCH_BYTES = 16 << 20
 

@@ -180,12 +180,9 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
       !stride_ok(out_stride_t) || !stride_ok(out_stride_h))
     return fail(QSA_ERR_INVALID_ARG, "tensor strides must be non-negative multiples of 8 elements");
   if (idx_stride_t < 0) return fail(QSA_ERR_INVALID_ARG, "negative idx_stride_t");
-  // The kernels address a gathered row by a 32-bit offset in 16-byte units: the
-  // largest slot's offset must fit (a 64 GiB reach per cache tensor).
-  const uint64_t last_slot = S > 0 ? uint64_t(S - 1) : 0;
-  if (last_slot * uint64_t(k_stride_s / 8) > UINT32_MAX ||
-      last_slot * uint64_t(v_stride_s / 8) > UINT32_MAX)
-    return fail(QSA_ERR_UNSUPPORTED, "cache extent beyond 64 GiB from its base");
+  // The kernels step from slot to slot by a 32-bit byte stride.
+  if (uint64_t(k_stride_s) * 2 > UINT32_MAX || uint64_t(v_stride_s) * 2 > UINT32_MAX)
+    return fail(QSA_ERR_UNSUPPORTED, "slot stride of 4 GiB or more");
 
   int32_t num_sms = 0;
   if (nsplit == 0) {
@@ -235,8 +232,8 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
   p.W = W;
   p.nsplit = pl.nsplit;
   p.split_len = pl.split_len;
-  p.k_row16 = uint32_t(k_stride_s / 8);
-  p.v_row16 = uint32_t(v_stride_s / 8);
+  p.k_row_bytes = uint32_t(k_stride_s * 2);
+  p.v_row_bytes = uint32_t(v_stride_s * 2);
   p.scale_log2 = scale * 1.4426950408889634f;  // log2(e): the kernels use 2^x
   p.block = block;
 

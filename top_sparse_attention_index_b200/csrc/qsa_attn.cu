@@ -52,26 +52,27 @@ struct Cfg {
   static constexpr int kStageBytes = SL * kSubBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;    // [slot lane][stage][sub-tile]
   static constexpr int kQBytes = NTILE * 8 * kRowBytes;
-  static constexpr int kIdxBytes = kMaxSlotsPerSplit * 8;  // (K, V) row offsets per slot
+  static constexpr int kIdxBytes = kMaxSlotsPerSplit * 4;  // compacted slot numbers
   static constexpr int kScanBytes = 32 * 4;
   static constexpr int kMergeBytes = kWarps * (8 * kMergeStride + 16) * 4;
   static constexpr size_t kSmem = size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes;
   static_assert(kMergeBytes <= kRingBytes, "merge buffer reuses the ring");
   static_assert(kMaxSlotsPerSplit * 4 <= kRingBytes, "raw index staging reuses the ring");
   static_assert(kMaxSlotsPerSplit % 16 == 0, "the offset list pads to whole sub-tiles");
+  // shared memory one SM gives its resident CTAs (228 KiB, 1 KiB reserved per CTA)
+  static constexpr size_t kSmPerCta(int ctas) { return 233472 / ctas - 1024; }
 };
 
-template <int NTILE, int SL, int STAGES>
-__global__ void __launch_bounds__(32 * NTILE * SL, 1)
+template <int NTILE, int SL, int STAGES, int MINB>
+__global__ void __launch_bounds__(32 * NTILE * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p) {
   using C = Cfg<NTILE, SL, STAGES>;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
   uint8_t* sQ = smem + C::kRingBytes;
-  // Compacted valid slots as row offsets in 16-byte units: (slot * k_stride_s / 8,
-  // slot * v_stride_s / 8); the host guarantees both fit in 32 bits.
-  uint2* sOff = reinterpret_cast<uint2*>(sQ + C::kQBytes);
-  int32_t* sScan = reinterpret_cast<int32_t*>(sOff + kMaxSlotsPerSplit);
+  // Compacted valid slot numbers of the split, padded to whole 16-slot sub-tiles.
+  uint32_t* sSlot = reinterpret_cast<uint32_t*>(sQ + C::kQBytes);
+  int32_t* sScan = reinterpret_cast<int32_t*>(sSlot + kMaxSlotsPerSplit);
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -141,12 +142,12 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
       if (v >= 0 && (int64_t(v) + 1) * block <= p.S) {
         for (int e = 0; e < block; ++e) {
           const uint32_t slot = uint32_t(v) * uint32_t(block) + uint32_t(e);
-          sOff[pos++] = make_uint2(slot * p.k_row16, slot * p.v_row16);
+          sSlot[pos++] = slot;
         }
       }
     }
   }
-  __syncthreads();  // sOff complete, the ring is free again
+  __syncthreads();  // sSlot complete, the ring is free again
 
   const int G = p.G;
   const int64_t head0 = int64_t(j) * G;
@@ -179,15 +180,17 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
   const int n_stages = (n_valid + C::kRows - 1) / C::kRows;
   // Pad the offset list to whole 16-slot sub-tiles with the first slot: padding rows
   // hold finite data and are masked out of the softmax.
-  for (int i = n_valid + tid; i < ((n_valid + 15) & ~15); i += C::kThreads) sOff[i] = sOff[0];
-  // Gather addressing: global-space row bases (one mad.wide per row and tensor in the
-  // loop) and, per lane, the eight swizzled chunk offsets (row & 7 is a compile-time
+  for (int i = n_valid + tid; i < ((n_valid + 15) & ~15); i += C::kThreads) sSlot[i] = sSlot[0];
+  // Gather addressing: global-space row bases, a row = base + slot * stride in bytes (one
+  // 32x32->64-bit mad per row and tensor in the loop) and, per lane, the eight swizzled
+  // chunk offsets (row & 7 is a compile-time
   // constant in the unrolled loop because a lane's rows start at 0 or 8), so a
   // destination is a register plus an immediate.
   const uint64_t kg = static_cast<uint64_t>(__cvta_generic_to_global(
                           p.k_cache + int64_t(j) * p.k_stride_h)) + uint64_t(lane) * 16;
   const uint64_t vg = static_cast<uint64_t>(__cvta_generic_to_global(
                           p.v_cache + int64_t(j) * p.v_stride_h)) + uint64_t(lane) * 16;
+  const uint32_t kstride = p.k_row_bytes, vstride = p.v_row_bytes;
   const uint32_t lane16 = uint32_t(lane) << 4;
   // this lane's sub-tiles: [wslot][stage]; a warp pair splits the 16 rows 8 / 8
   const uint32_t sub_s = ring_s + wslot * STAGES * C::kSubBytes;
@@ -201,16 +204,17 @@ __global__ void __launch_bounds__(32 * NTILE * SL, 1)
     uint32_t kd[8];
 #pragma unroll
     for (int m = 0; m < 8; ++m) kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (m << 4));
-    const uint4* offs = reinterpret_cast<const uint4*>(sOff + base + row0);  // 16-byte aligned
+    const uint4* slots = reinterpret_cast<const uint4*>(sSlot + base + row0);  // 16-byte aligned
 #pragma unroll
-    for (int i = 0; i < kLoadRows; i += 2) {
-      const uint4 o2 = offs[i / 2];  // offsets of rows i and i + 1
-      const uint32_t d0 = kd[i & 7] + i * kRowBytes;
-      const uint32_t d1 = kd[(i + 1) & 7] + (i + 1) * kRowBytes;
-      cp_async_16_global(d0, kg + uint64_t(o2.x) * 16);
-      cp_async_16_global(d0 + 16 * kRowBytes, vg + uint64_t(o2.y) * 16);
-      cp_async_16_global(d1, kg + uint64_t(o2.z) * 16);
-      cp_async_16_global(d1 + 16 * kRowBytes, vg + uint64_t(o2.w) * 16);
+    for (int i = 0; i < kLoadRows; i += 4) {
+      const uint4 s4 = slots[i / 4];  // slots of rows i .. i + 3
+      const uint32_t sl[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t d = kd[(i + e) & 7] + (i + e) * kRowBytes;
+        cp_async_16_global(d, kg + uint64_t(sl[e]) * kstride);
+        cp_async_16_global(d + 16 * kRowBytes, vg + uint64_t(sl[e]) * vstride);
+      }
     }
   };
   // makes a stage's sub-tile, loaded by one warp or a warp pair, visible to it
@@ -459,10 +463,10 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
   *dst = v;
 }
 
-template <int NTILE, int SL, int STAGES>
+template <int NTILE, int SL, int STAGES, int MINB>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
   using C = Cfg<NTILE, SL, STAGES>;
-  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, SL, STAGES>;
+  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, SL, STAGES, MINB>;
   // The shared-memory opt-in is a per-device function attribute: set it on the first
   // launch on each device only, so later calls (e.g. under stream capture) are launches
   // and nothing else.
@@ -482,30 +486,41 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// The two shapes (slot lanes x pipeline stages per lane, chosen by measurement):
-// G <= 8: one n8 tile, QSA_SMALL_SL slot lanes of one warp each;
-// 8 < G <= 16: two n8 tiles, QSA_LARGE_SL slot lanes of a warp pair each.
+// The two shapes (slot lanes x pipeline stages per lane x resident CTAs per SM, chosen by
+// measurement): G <= 8: one n8 tile, slot lanes of one warp each; 8 < G <= 16: two n8
+// tiles, slot lanes of a warp pair each.  Two CTAs per SM hide each other's prologue
+// (index compaction, Q load, pipeline fill) and epilogue (warp merge, output write).
 #ifndef QSA_SMALL_SL
-#define QSA_SMALL_SL 6
+#define QSA_SMALL_SL 3
 #endif
 #ifndef QSA_SMALL_STAGES
 #define QSA_SMALL_STAGES 2
 #endif
+#ifndef QSA_SMALL_CTAS
+#define QSA_SMALL_CTAS 2  // CTAs resident per SM
+#endif
 #ifndef QSA_LARGE_SL
-#define QSA_LARGE_SL 6
+#define QSA_LARGE_SL 3
 #endif
 #ifndef QSA_LARGE_STAGES
 #define QSA_LARGE_STAGES 2
 #endif
+#ifndef QSA_LARGE_CTAS
+#define QSA_LARGE_CTAS 2
+#endif
 using CfgSmall = Cfg<1, QSA_SMALL_SL, QSA_SMALL_STAGES>;
 using CfgLarge = Cfg<2, QSA_LARGE_SL, QSA_LARGE_STAGES>;
+static_assert(CfgSmall::kSmem <= CfgSmall::kSmPerCta(QSA_SMALL_CTAS), "small shape: CTAs per SM");
+static_assert(CfgLarge::kSmem <= CfgLarge::kSmPerCta(QSA_LARGE_CTAS), "large shape: CTAs per SM");
 
 }  // namespace
 
 KernelShape kernel_shape(int G) {
   if (G <= 8)
-    return {1, QSA_SMALL_SL, CfgSmall::kThreads, CfgSmall::kRows, QSA_SMALL_STAGES, CfgSmall::kSmem, 1};
-  return {2, QSA_LARGE_SL, CfgLarge::kThreads, CfgLarge::kRows, QSA_LARGE_STAGES, CfgLarge::kSmem, 1};
+    return {1, QSA_SMALL_SL, CfgSmall::kThreads, CfgSmall::kRows, QSA_SMALL_STAGES, CfgSmall::kSmem,
+            QSA_SMALL_CTAS};
+  return {2, QSA_LARGE_SL, CfgLarge::kThreads, CfgLarge::kRows, QSA_LARGE_STAGES, CfgLarge::kSmem,
+          QSA_LARGE_CTAS};
 }
 
 size_t workspace_lse_offset(int32_t Tq, int32_t Hq, int32_t nsplit) {
@@ -520,8 +535,9 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
 }
 
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = (p.G <= 8) ? launch_fwd<1, QSA_SMALL_SL, QSA_SMALL_STAGES>(p, stream)
-                             : launch_fwd<2, QSA_LARGE_SL, QSA_LARGE_STAGES>(p, stream);
+  cudaError_t e = (p.G <= 8)
+                      ? launch_fwd<1, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS>(p, stream)
+                      : launch_fwd<2, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS>(p, stream);
   if (e != cudaSuccess || p.nsplit == 1) return e;
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);

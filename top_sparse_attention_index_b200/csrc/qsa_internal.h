@@ -11,7 +11,7 @@ namespace qsa {
 
 constexpr int kHeadDim = 256;           // D: the only head dimension implemented
 constexpr int kMaxGroup = 16;           // largest G = Hq / Hkv
-constexpr int kMaxSlotsPerSplit = 2560; // per-split index list staged in shared memory
+constexpr int kMaxSlotsPerSplit = 2240; // per-split slot list staged in shared memory
 constexpr int kMinSlotsPerSplit = 128;  // the planner never makes splits narrower
 constexpr int kMaxBlock = 16;           // largest block size of block selection
 
@@ -35,8 +35,8 @@ struct FwdParams {
   int32_t Tq, Hq, Hkv, G, W;
   int32_t nsplit;
   int32_t split_len;        // positions of the W axis per split
-  uint32_t k_row16;         // k_stride_s / 8: one slot step of K in 16-byte units
-  uint32_t v_row16;         // v_stride_s / 8
+  uint32_t k_row_bytes;     // k_stride_s * 2: one slot step of K in bytes
+  uint32_t v_row_bytes;     // v_stride_s * 2
   float scale_log2;         // scale * log2(e)
   int32_t block;            // slots named by one selected entry (1 = slot selection)
 };

@@ -11,7 +11,10 @@ namespace qsa {
 
 constexpr int kHeadDim = 256;           // D: the only head dimension implemented
 constexpr int kMaxGroup = 16;           // largest G = Hq / Hkv
-constexpr int kMaxSlotsPerSplit = 2240; // per-split slot list staged in shared memory
+#ifndef QSA_MAX_SLOTS
+#define QSA_MAX_SLOTS 2240
+#endif
+constexpr int kMaxSlotsPerSplit = QSA_MAX_SLOTS;  // per-split slot list staged in smem
 constexpr int kMinSlotsPerSplit = 128;  // the planner never makes splits narrower
 constexpr int kMaxBlock = 16;           // largest block size of block selection
 

@@ -302,24 +302,29 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
     }
     float x0 = (sa[0] + sb[0]) * sl2, x1 = (sa[1] + sb[1]) * sl2;
     float x2 = (sa[2] + sb[2]) * sl2, x3 = (sa[3] + sb[3]) * sl2;
-    const int r0 = base + (lane >> 2);
-    if (r0 >= n_valid) x0 = x1 = kNegInf;
-    if (r0 + 8 >= n_valid) x2 = x3 = kNegInf;
-
-    // online softmax over the slot axis (rows): lanes sharing l%4 hold one head pair
-    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    if (base + 16 > n_valid) {  // warp-uniform: only the last sub-tile has padding rows
+      const int r0 = base + (lane >> 2);
+      if (r0 >= n_valid) x0 = x1 = kNegInf;
+      if (r0 + 8 >= n_valid) x2 = x3 = kNegInf;
     }
+
+    // Online softmax over the slot axis (rows); lanes sharing l%4 hold one head pair.
     // Lazy rescaling: the reference max m only moves when the chunk max exceeds it by
     // more than kRescaleLog2 (weights stay <= 2^kRescaleLog2, exact in fp32 and within
     // bf16 range); the final normalisation uses the same m for O and l, so the result
-    // is unchanged.  mx is finite here: row `base` of this sub-tile is valid.
-    const float mn0 = (mx0 > m0 + kRescaleLog2) ? mx0 : m0;
-    const float mn1 = (mx1 > m1 + kRescaleLog2) ? mx1 : m1;
-    if (__any_sync(0xffffffffu, mn0 != m0 || mn1 != m1)) {
+    // is unchanged.  A vote on the lanes' own maxima decides whether any head moves;
+    // only then is the exact chunk max reduced over the slot axis (the decision is the
+    // same as comparing the exact max).  The max is finite: row `base` is valid.
+    const float lx0 = fmaxf(x0, x2), lx1 = fmaxf(x1, x3);
+    if (__any_sync(0xffffffffu, lx0 > m0 + kRescaleLog2 || lx1 > m1 + kRescaleLog2)) {
+      float mx0 = lx0, mx1 = lx1;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = (mx0 > m0 + kRescaleLog2) ? mx0 : m0;
+      const float mn1 = (mx1 > m1 + kRescaleLog2) ? mx1 : m1;
       const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);  // -inf -> 0
       l0 *= al0;
       l1 *= al1;

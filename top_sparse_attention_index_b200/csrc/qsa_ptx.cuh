@@ -23,11 +23,6 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool 
                : "memory");
 }
 
-// 16-byte async copy global -> shared, always reading the source.
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-}
-
 // 16-byte async copy from a global-space address (from __cvta_generic_to_global).
 __device__ __forceinline__ void cp_async_16_global(uint32_t dst, uint64_t gaddr) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(gaddr) : "memory");

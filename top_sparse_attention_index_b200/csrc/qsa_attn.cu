@@ -43,9 +43,10 @@ constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent)
 
 
-template <int NTILE, int SL, int STAGES>
+template <int NTILE, int DSPLIT, int SL, int STAGES>
 struct Cfg {
-  static constexpr int kWarps = NTILE * SL;
+  static constexpr int kParts = NTILE * DSPLIT;  // warps serving one slot lane
+  static constexpr int kWarps = kParts * SL;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kRows = 16 * SL;                      // slots per stage
   static constexpr int kSubBytes = 16 * kRowBytes * 2;       // one sub-tile: 16 K rows, 16 V rows
@@ -63,10 +64,15 @@ struct Cfg {
   static constexpr size_t kSmPerCta(int ctas) { return 233472 / ctas - 1024; }
 };
 
-template <int NTILE, int SL, int STAGES, int MINB>
-__global__ void __launch_bounds__(32 * NTILE * SL, MINB)
+// NTILE n8 tiles cover the head group (G <= 8: 1; G <= 16: 2).  The warps of one slot
+// lane split either the head tiles (NTILE = 2) or, with DSPLIT = 2, the D rows of the PV
+// product (both compute the same scores).
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB>
+__global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p) {
-  using C = Cfg<NTILE, SL, STAGES>;
+  static_assert(NTILE == 1 || DSPLIT == 1, "a lane splits either the heads or D");
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES>;
+  constexpr int kMT = 16 / DSPLIT;  // m16 tiles of D per warp in the PV product
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
   uint8_t* sQ = smem + C::kRingBytes;
@@ -78,7 +84,9 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int wslot = warp % SL;  // which 16-slot sub-tile of a stage
-  const int wn = warp / SL;     // which n8 tile of the head group
+  const int wpart = warp / SL;             // which warp of the slot lane
+  const int wn = NTILE > 1 ? wpart : 0;    // which n8 tile of the head group
+  const int wd = DSPLIT > 1 ? wpart : 0;   // which D range of the PV product
 
   // ---- work unit -------------------------------------------------------------------
   int u = blockIdx.x;
@@ -194,8 +202,8 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
   const uint32_t lane16 = uint32_t(lane) << 4;
   // this lane's sub-tiles: [wslot][stage]; a warp pair splits the 16 rows 8 / 8
   const uint32_t sub_s = ring_s + wslot * STAGES * C::kSubBytes;
-  constexpr int kLoadRows = 16 / NTILE;
-  const int row0 = wn * kLoadRows;
+  constexpr int kLoadRows = 16 / C::kParts;
+  const int row0 = wpart * kLoadRows;
   const uint32_t sub_rows = sub_s + row0 * kRowBytes;
 
   auto load_stage = [&](int s, int buf) {
@@ -219,10 +227,10 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
   };
   // makes a stage's sub-tile, loaded by one warp or a warp pair, visible to it
   auto lane_sync = [&]() {
-    if constexpr (NTILE == 1) {
+    if constexpr (C::kParts == 1) {
       __syncwarp();
     } else {
-      named_barrier_sync(1 + wslot, 32 * NTILE);
+      named_barrier_sync(1 + wslot, 32 * C::kParts);
     }
   };
   __syncthreads();  // the padded offset list is complete
@@ -252,9 +260,9 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
   // ---- 3. main loop ------------------------------------------------------------------
   float m0 = kNegInf, m1 = kNegInf;  // reference max (base 2) of heads 2(l%4), 2(l%4)+1
   float l0 = 0.f, l1 = 0.f;          // this lane's share of the running sums
-  float o[16][4];
+  float o[kMT][4];
 #pragma unroll
-  for (int mt = 0; mt < 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  for (int mt = 0; mt < kMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
 
   // ldmatrix addressing.  Chunk c of a row sits at ((c ^ key) << 4), key = row & 7 =
   // lane & 7 for every row this lane addresses.  With c = 2 * step + hi (step = k-step
@@ -329,7 +337,7 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
       l0 *= al0;
       l1 *= al1;
 #pragma unroll
-      for (int mt = 0; mt < 16; ++mt) {
+      for (int mt = 0; mt < kMT; ++mt) {
         o[mt][0] *= al0;
         o[mt][1] *= al1;
         o[mt][2] *= al0;
@@ -344,14 +352,14 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
     l0 += bf16lo_to_f32(p01) + bf16lo_to_f32(p23);
     l1 += bf16hi_to_f32(p01) + bf16hi_to_f32(p23);
 
-    // O^T (256 x 8) += V^T (256 x 16) * P^T (16 x 8)
+    // O^T (this warp's D rows x 8) += V^T (D rows x 16) * P^T (16 x 8)
     const uint32_t b0 = movmatrix_trans(p01);
     const uint32_t b1 = movmatrix_trans(p23);
     uint32_t vt[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m];
+    for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / 4) * 128;
 #pragma unroll
-    for (int mt = 0; mt < 16; ++mt) {
+    for (int mt = 0; mt < kMT; ++mt) {
       uint32_t a[4];
       ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
       mma_bf16_16816(o[mt], a, b0, b1);
@@ -373,8 +381,8 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
     const int g0 = 2 * (lane & 3);
     const int r8 = lane >> 2;
 #pragma unroll
-    for (int mt = 0; mt < 16; ++mt) {
-      const int d = 16 * mt + r8;
+    for (int mt = 0; mt < kMT; ++mt) {
+      const int d = 16 * (wd * kMT + mt) + r8;
       mine[g0 * kMergeStride + d] = o[mt][0];
       mine[(g0 + 1) * kMergeStride + d] = o[mt][1];
       mine[g0 * kMergeStride + d + 8] = o[mt][2];
@@ -394,17 +402,19 @@ __global__ void __launch_bounds__(32 * NTILE * SL, MINB)
     const int dg = it & 31;  // 8-wide d group
     if (gg >= G) continue;
     const int nt = gg >> 3, g = gg & 7;
+    // the warps holding this (head, d) range: one per slot lane
+    const int part = NTILE > 1 ? nt : (dg * 8) / (kHeadDim / DSPLIT);
     float mstar = kNegInf;
 #pragma unroll
     for (int w = 0; w < SL; ++w)
-      mstar = fmaxf(mstar, mbuf[(nt * SL + w) * kWarpFloats + 8 * kMergeStride + g]);
+      mstar = fmaxf(mstar, mbuf[(part * SL + w) * kWarpFloats + 8 * kMergeStride + g]);
     float lsum = 0.f;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
     for (int w = 0; w < SL; ++w) {
-      const float* src = mbuf + (nt * SL + w) * kWarpFloats;
+      const float* src = mbuf + (part * SL + w) * kWarpFloats;
       const float sc = fast_exp2(src[8 * kMergeStride + g] - mstar);  // -inf -> 0
       lsum += sc * src[8 * kMergeStride + 8 + g];
       const float4 a = *reinterpret_cast<const float4*>(src + g * kMergeStride + dg * 8);
@@ -468,10 +478,10 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
   *dst = v;
 }
 
-template <int NTILE, int SL, int STAGES, int MINB>
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
-  using C = Cfg<NTILE, SL, STAGES>;
-  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, SL, STAGES, MINB>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES>;
+  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB>;
   // The shared-memory opt-in is a per-device function attribute: set it on the first
   // launch on each device only, so later calls (e.g. under stream capture) are launches
   // and nothing else.
@@ -513,8 +523,11 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
 #ifndef QSA_LARGE_CTAS
 #define QSA_LARGE_CTAS 2
 #endif
-using CfgSmall = Cfg<1, QSA_SMALL_SL, QSA_SMALL_STAGES>;
-using CfgLarge = Cfg<2, QSA_LARGE_SL, QSA_LARGE_STAGES>;
+#ifndef QSA_SMALL_DSPLIT
+#define QSA_SMALL_DSPLIT 2
+#endif
+using CfgSmall = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES>;
+using CfgLarge = Cfg<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES>;
 static_assert(CfgSmall::kSmem <= CfgSmall::kSmPerCta(QSA_SMALL_CTAS), "small shape: CTAs per SM");
 static_assert(CfgLarge::kSmem <= CfgLarge::kSmPerCta(QSA_LARGE_CTAS), "large shape: CTAs per SM");
 
@@ -541,8 +554,9 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
 
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   cudaError_t e = (p.G <= 8)
-                      ? launch_fwd<1, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS>(p, stream)
-                      : launch_fwd<2, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS>(p, stream);
+                      ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES,
+                                   QSA_SMALL_CTAS>(p, stream)
+                      : launch_fwd<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS>(p, stream);
   if (e != cudaSuccess || p.nsplit == 1) return e;
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);

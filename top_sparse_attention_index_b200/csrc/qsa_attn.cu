@@ -6,21 +6,23 @@
 // scale * Q K^T for the whole GQA group of G = Hq / Hkv query heads, take the softmax
 // over the selected slots only and return P V; a row without a valid slot returns 0.
 //
-// K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit:
+// K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit, two CTAs
+// resident per SM so that one CTA's prologue and epilogue overlap the other's gather:
 //   1. stage the split's slot indices in shared memory and compact away -1 (and
 //      out-of-range) entries with a block scan, so masked slots cost no bandwidth;
 //   2. gather K and V rows of the compacted slots with 16-byte cp.async into shared
-//      memory: each 16-slot sub-tile of a stage belongs to one slot lane (one warp, or a
-//      warp pair when G > 8) that loads it, waits for it and consumes it, so the lanes
-//      run STAGES-deep pipelines of their own with no block-wide barrier in the loop
-//      (row = 512 contiguous bytes; the 16-byte chunks of a row are XOR-swizzled by the
-//      row index so ldmatrix reads are conflict-free);
-//   3. per warp and 16-slot sub-tile: S^T = K Q^T with the slots as the MMA M dimension
-//      and the (up to 8) heads of one n8 tile as N, so the group shares every gathered
-//      row and G = 3/6/8/12/16 needs no padding of the head ratio in memory;
-//      online softmax in fp32 registers (base 2, warp shuffles over the slot axis);
-//      P rounded to bf16 and transposed in registers (movmatrix) into the B operand of
-//      O^T += V^T P^T with D = 256 as M;
+//      memory: each 16-slot sub-tile of a stage belongs to one slot lane (a warp pair)
+//      that loads it, waits for it and consumes it, so the lanes run STAGES-deep
+//      pipelines of their own with no block-wide barrier in the loop (row = 512
+//      contiguous bytes; the 16-byte chunks of a row are XOR-swizzled by the row index
+//      so ldmatrix reads are conflict-free);
+//   3. per slot lane and 16-slot sub-tile: S^T = K Q^T with the slots as the MMA M
+//      dimension and the (up to 8) heads of one n8 tile as N, so the group shares every
+//      gathered row and G = 3/6/8/12/16 needs no padding of the head ratio in memory
+//      (G <= 8: the pair splits D for both products and exchanges partial scores;
+//      G > 8: the pair splits the two head tiles); online softmax in fp32 registers
+//      (base 2, lazy rescaling); P rounded to bf16 and transposed in registers
+//      (movmatrix) into the B operand of O^T += V^T P^T with D = 256 as M;
 //   4. merge the per-warp (m, l, O) states through shared memory and write bf16 out
 //      (exact zeros for empty rows), or fp32 partials + base-2 LSE when split.
 // K2 qsa_lse_combine_kernel -- one warp per (t, h): log-sum-exp weighted sum of the
@@ -55,8 +57,11 @@ struct Cfg {
   static constexpr int kQBytes = NTILE * 8 * kRowBytes;
   static constexpr int kIdxBytes = kMaxSlotsPerSplit * 4;  // compacted slot numbers
   static constexpr int kScanBytes = 32 * 4;
+  // partial scores a D-split pair exchanges when it also splits Q K^T: [lane][warp][32][4]
+  static constexpr int kXchgBytes = (DSPLIT > 1) ? SL * DSPLIT * 32 * 16 : 0;
   static constexpr int kMergeBytes = kWarps * (8 * kMergeStride + 16) * 4;
-  static constexpr size_t kSmem = size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes;
+  static constexpr size_t kSmem =
+      size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes + kXchgBytes;
   static_assert(kMergeBytes <= kRingBytes, "merge buffer reuses the ring");
   static_assert(kMaxSlotsPerSplit * 4 <= kRingBytes, "raw index staging reuses the ring");
   static_assert(kMaxSlotsPerSplit % 16 == 0, "the offset list pads to whole sub-tiles");
@@ -67,10 +72,12 @@ struct Cfg {
 // NTILE n8 tiles cover the head group (G <= 8: 1; G <= 16: 2).  The warps of one slot
 // lane split either the head tiles (NTILE = 2) or, with DSPLIT = 2, the D rows of the PV
 // product (both compute the same scores).
-template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB>
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT>
 __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p) {
   static_assert(NTILE == 1 || DSPLIT == 1, "a lane splits either the heads or D");
+  static_assert(!QSPLIT || DSPLIT == 2, "splitting Q K^T needs a D-split pair");
+  constexpr int kKS = QSPLIT ? 8 : 16;  // k-steps of Q K^T per warp
   using C = Cfg<NTILE, DSPLIT, SL, STAGES>;
   constexpr int kMT = 16 / DSPLIT;  // m16 tiles of D per warp in the PV product
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -79,6 +86,7 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
   // Compacted valid slot numbers of the split, padded to whole 16-slot sub-tiles.
   uint32_t* sSlot = reinterpret_cast<uint32_t*>(sQ + C::kQBytes);
   int32_t* sScan = reinterpret_cast<int32_t*>(sSlot + kMaxSlotsPerSplit);
+  float4* sXchg = reinterpret_cast<float4*>(sScan + 32);  // (DSPLIT > 1 and QSPLIT only)
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -86,7 +94,8 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
   const int wslot = warp % SL;  // which 16-slot sub-tile of a stage
   const int wpart = warp / SL;             // which warp of the slot lane
   const int wn = NTILE > 1 ? wpart : 0;    // which n8 tile of the head group
-  const int wd = DSPLIT > 1 ? wpart : 0;   // which D range of the PV product
+  const int wd = DSPLIT > 1 ? wpart : 0;   // which D range of the PV product (and of
+                                           // Q K^T with QSPLIT)
 
   // ---- work unit -------------------------------------------------------------------
   int u = blockIdx.x;
@@ -244,11 +253,13 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
   __syncthreads();
 
   // B fragments of Q^T for this warp's n8 tile, all 16 k-steps of D = 256.
-  uint32_t qf[16][2];
+  // (with QSPLIT, warp wd of a pair keeps the k-steps of its half of D only)
+  uint32_t qf[kKS][2];
+  const int ks0 = QSPLIT ? wd * kKS : 0;
 #pragma unroll
-  for (int kp = 0; kp < 8; ++kp) {
+  for (int kp = 0; kp < kKS / 2; ++kp) {
     const int g = lane & 7;
-    const int c = 4 * kp + (lane >> 3);
+    const int c = 4 * kp + 2 * ks0 + (lane >> 3);
     uint32_t r[4];
     ldmatrix_x4(r, q_s + (wn * 8 + g) * kRowBytes + ((c ^ g) << 4));
     qf[2 * kp][0] = r[0];
@@ -298,18 +309,33 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8); two chains for ILP.
     uint32_t kt[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) kt[m] = sub + kswz[m];
+    for (int m = 0; m < 4; ++m) kt[m] = sub + kswz[m] + ks0 * 32;  // 16 k-steps = 4 x 128 B
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int ks = 0; ks < 16; ks += 2) {
+    for (int ks = 0; ks < kKS; ks += 2) {
       uint32_t a[4];
       ldmatrix_x4(a, kt[ks & 3] + 128 * (ks >> 2));
       mma_bf16_16816(sa, a, qf[ks][0], qf[ks][1]);
       ldmatrix_x4(a, kt[(ks + 1) & 3] + 128 * ((ks + 1) >> 2));
       mma_bf16_16816(sb, a, qf[ks + 1][0], qf[ks + 1][1]);
     }
-    float x0 = (sa[0] + sb[0]) * sl2, x1 = (sa[1] + sb[1]) * sl2;
-    float x2 = (sa[2] + sb[2]) * sl2, x3 = (sa[3] + sb[3]) * sl2;
+    float s0 = sa[0] + sb[0], s1 = sa[1] + sb[1], s2 = sa[2] + sb[2], s3 = sa[3] + sb[3];
+    if constexpr (QSPLIT) {
+      // each warp of the pair holds the scores over its half of D: exchange and add in
+      // a fixed order (low half + high half) so both warps hold the same scores
+      float4* mine = sXchg + (wslot * 2 + wd) * 32 + lane;
+      float4* other = sXchg + (wslot * 2 + (wd ^ 1)) * 32 + lane;
+      *mine = make_float4(s0, s1, s2, s3);
+      named_barrier_sync(1 + wslot, 64);
+      const float4 t = *other;
+      if (wd == 0) {
+        s0 += t.x; s1 += t.y; s2 += t.z; s3 += t.w;
+      } else {
+        s0 = t.x + s0; s1 = t.y + s1; s2 = t.z + s2; s3 = t.w + s3;
+      }
+    }
+    float x0 = s0 * sl2, x1 = s1 * sl2;
+    float x2 = s2 * sl2, x3 = s3 * sl2;
     if (base + 16 > n_valid) {  // warp-uniform: only the last sub-tile has padding rows
       const int r0 = base + (lane >> 2);
       if (r0 >= n_valid) x0 = x1 = kNegInf;
@@ -478,10 +504,10 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
   *dst = v;
 }
 
-template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB>
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
   using C = Cfg<NTILE, DSPLIT, SL, STAGES>;
-  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB>;
+  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT>;
   // The shared-memory opt-in is a per-device function attribute: set it on the first
   // launch on each device only, so later calls (e.g. under stream capture) are launches
   // and nothing else.
@@ -526,6 +552,9 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
 #ifndef QSA_SMALL_DSPLIT
 #define QSA_SMALL_DSPLIT 2
 #endif
+#ifndef QSA_SMALL_QSPLIT
+#define QSA_SMALL_QSPLIT true
+#endif
 using CfgSmall = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES>;
 using CfgLarge = Cfg<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES>;
 static_assert(CfgSmall::kSmem <= CfgSmall::kSmPerCta(QSA_SMALL_CTAS), "small shape: CTAs per SM");
@@ -555,8 +584,9 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   cudaError_t e = (p.G <= 8)
                       ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES,
-                                   QSA_SMALL_CTAS>(p, stream)
-                      : launch_fwd<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS>(p, stream);
+                                   QSA_SMALL_CTAS, QSA_SMALL_QSPLIT>(p, stream)
+                      : launch_fwd<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS, false>(
+                            p, stream);
   if (e != cudaSuccess || p.nsplit == 1) return e;
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);

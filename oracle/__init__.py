@@ -53,6 +53,14 @@ class Oracle:
         fb.restype = ctypes.c_int
         fb.argtypes = [p, i64, i64, p, i64, i64, p, i64, i64, p, i64, p,
                        i32, i32, i32, i32, i64, i32, i32, ctypes.c_float, p, i64, p, p]
+        f8 = self._lib.qsa_oracle_forward_fp8kv
+        f8.restype = ctypes.c_int
+        f8.argtypes = [p, i64, i64, p, i64, i64, p, i64, i64, p, i64, p,
+                       i32, i32, i32, i32, i64, i32, i32, ctypes.c_float, ctypes.c_float,
+                       ctypes.c_float, p, i64, p, p]
+        dec = self._lib.qsa_oracle_decode_e4m3
+        dec.restype = None
+        dec.argtypes = [p, i64, p]
         self._lib.qsa_oracle_num_threads.restype = ctypes.c_int
         self.path = path
 
@@ -103,6 +111,65 @@ class Oracle:
         if rc != 0:
             raise ValueError("oracle rejected the sizes")
         return (out, int(err.value)) if return_err else out
+
+
+    def decode_e4m3(self, codes) -> np.ndarray:
+        """float32 values of E4M3 codes (uint8 array or float8_e4m3fn / uint8 tensor)."""
+        c = np.ascontiguousarray(_as_u8(codes))
+        out = np.empty(c.shape, dtype=np.float32)
+        self._lib.qsa_oracle_decode_e4m3(c.ctypes.data, c.size, out.ctypes.data)
+        return out
+
+    def forward_fp8kv(self, q, k_cache, v_cache, slot_idx, width=None, scale=1.0 / 16.0,
+                      k_scale=1.0, v_scale=1.0, rows=None, S=None, return_err=False, block=1):
+        """fp32 oracle output with an fp8_e4m3 K/V cache.
+
+        k_cache / v_cache: E4M3 codes [S, Hkv, D] as a uint8 array or a float8_e4m3fn /
+        uint8 CPU tensor (d contiguous); a dequantised element is its code's value times
+        k_scale (v_scale).  Everything else as ``forward``.
+        """
+        q = _as_bf16_bits(q)
+        k_cache, v_cache = _as_u8(k_cache), _as_u8(v_cache)
+        slot_idx = _as_i32(slot_idx)
+        Tq, Hq, D = q.shape
+        S_, Hkv, Dk = k_cache.shape
+        assert Dk == D and v_cache.shape == k_cache.shape
+        S = S_ if S is None else S
+        W = slot_idx.shape[1]
+        assert q.strides[-1] == 2 and k_cache.strides[-1] == 1 and v_cache.strides[-1] == 1
+        assert slot_idx.strides[1] == 4
+        if width is not None:
+            width = np.ascontiguousarray(_as_i32(width))
+            assert width.shape == (Tq,)
+        if rows is not None:
+            rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+            nrows = rows.shape[0]
+        else:
+            nrows = Tq
+        out = np.zeros((nrows, Hq, D), dtype=np.float32)
+        err = ctypes.c_uint32(0)
+        rc = self._lib.qsa_oracle_forward_fp8kv(
+            q.ctypes.data, q.strides[0] // 2, q.strides[1] // 2,
+            k_cache.ctypes.data, k_cache.strides[0], k_cache.strides[1],
+            v_cache.ctypes.data, v_cache.strides[0], v_cache.strides[1],
+            slot_idx.ctypes.data, slot_idx.strides[0] // 4,
+            None if width is None else width.ctypes.data, Tq, Hq, Hkv, D, S, W, block,
+            ctypes.c_float(scale), ctypes.c_float(k_scale), ctypes.c_float(v_scale),
+            None if rows is None else rows.ctypes.data, nrows, out.ctypes.data,
+            ctypes.byref(err))
+        if rc != 0:
+            raise ValueError("oracle rejected the sizes")
+        return (out, int(err.value)) if return_err else out
+
+
+def _as_u8(x) -> np.ndarray:
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint8
+        return x
+    import torch
+    assert isinstance(x, torch.Tensor) and x.device.type == "cpu"
+    assert x.dtype in (torch.uint8, torch.float8_e4m3fn)
+    return _strided_view(x.view(torch.uint8), np.uint8)
 
 
 def _as_bf16_bits(x) -> np.ndarray:

@@ -217,6 +217,137 @@ int qsa_oracle_forward_block(const uint16_t* q, int64_t q_stride_t, int64_t q_st
   return 0;
 }
 
+/*
+ * fp8_e4m3 KV cache.  The article's section "Where this sits in the Qwen4Exp serving
+ * build-out" reports fp8_e4m3 as the better-performing KV-cache format for this
+ * attention's decode.  Reading used here: the cache holds one OCP FP8 E4M3 code per
+ * element, and each of K and V carries one float scale (a dequantised element is
+ * code value x scale); the attention is then the definition above applied to the
+ * dequantised rows.
+ *
+ * e4m3_value -- the value of one E4M3 code, decoded field by field: 1 sign bit, 4
+ * exponent bits with bias 7, 3 mantissa bits; an exponent field of 0 encodes the
+ * subnormals (m / 8) * 2^(1 - 7); the pattern S.1111.111 is NaN and there are no
+ * infinities (the "FN" variant, largest finite magnitude 448).
+ */
+static float e4m3_value(uint8_t code) {
+  const int sign = code >> 7;
+  const int e = (code >> 3) & 15;
+  const int m = code & 7;
+  float mag;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    mag = ldexpf((float)m / 8.0f, 1 - 7);
+  else
+    mag = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+  return sign ? -mag : mag;
+}
+
+/* Decode n E4M3 codes (exported for the tests). */
+void qsa_oracle_decode_e4m3(const uint8_t* codes, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(codes[i]);
+}
+
+/*
+ * qsa_oracle_forward_fp8kv -- fp32 reference with an fp8_e4m3 K/V cache.
+ *   k_cache, v_cache  E4M3 codes, element (s, j, d) at k_cache[s*k_stride_s +
+ *                     j*k_stride_h + d] (strides in elements = bytes)
+ *   k_scale, v_scale  dequantisation scales: K = e4m3_value(code) * k_scale, likewise V
+ *   block             as qsa_oracle_forward_block (1 = slot selection)
+ * Every other argument as qsa_oracle_forward.  Steps per (t, KV head j): the valid
+ * selected slots (width, -1 and range rules of the slot-level definition, blocks
+ * expanded), their K and V rows dequantised into float, then for each query head of
+ * the group: scores scale * <q, k_i>, softmax over the selected slots, P V.
+ */
+int qsa_oracle_forward_fp8kv(const uint16_t* q, int64_t q_stride_t, int64_t q_stride_h,
+                             const uint8_t* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                             const uint8_t* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                             const int32_t* slot_idx, int64_t idx_stride_t, const int32_t* width,
+                             int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int64_t S, int32_t W,
+                             int32_t block, float scale, float k_scale, float v_scale,
+                             const int64_t* rows, int64_t nrows, float* out, uint32_t* err_bits) {
+  if (Tq < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || S < 0 || W < 0 || block < 1) return -1;
+  if (Hq % Hkv != 0) return -1;
+  const int32_t G = Hq / Hkv;
+  const int64_t n_out = rows ? nrows : (int64_t)Tq;
+  const int64_t cap = (int64_t)W * block;
+  const size_t cap1 = (size_t)(cap > 0 ? cap : 1);
+  uint32_t all_bits = 0;
+
+#pragma omp parallel reduction(| : all_bits)
+  {
+    int64_t* sel = (int64_t*)malloc(sizeof(int64_t) * cap1);
+    float* kf = (float*)malloc(sizeof(float) * cap1 * (size_t)D);
+    float* vf = (float*)malloc(sizeof(float) * cap1 * (size_t)D);
+    float* sc = (float*)malloc(sizeof(float) * cap1);
+    uint32_t bits = 0;
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n_out; ++r) {
+      const int64_t t = rows ? rows[r] : r;
+      int32_t width_t = width ? width[t] : W;
+      if (width_t < 0 || width_t > W) {
+        bits |= 2u;
+        width_t = width_t < 0 ? 0 : W;
+      }
+      /* 1. the valid selected slots of the row (blocks expanded, -1 skipped) */
+      const int32_t* idx_row = slot_idx + t * idx_stride_t;
+      int64_t n = 0;
+      for (int32_t w = 0; w < width_t; ++w) {
+        const int32_t b = idx_row[w];
+        if (b == -1) continue;
+        if (b < -1 || ((int64_t)b + 1) * block > S) {
+          bits |= 1u;
+          continue;
+        }
+        for (int32_t e = 0; e < block; ++e) sel[n++] = (int64_t)b * block + e;
+      }
+      for (int32_t j = 0; j < Hkv; ++j) {
+        /* 2. dequantise the selected K and V rows of KV head j */
+        for (int64_t i = 0; i < n; ++i) {
+          const uint8_t* k_row = k_cache + sel[i] * k_stride_s + (int64_t)j * k_stride_h;
+          const uint8_t* v_row = v_cache + sel[i] * v_stride_s + (int64_t)j * v_stride_h;
+          for (int32_t d = 0; d < D; ++d) {
+            kf[i * D + d] = e4m3_value(k_row[d]) * k_scale;
+            vf[i * D + d] = e4m3_value(v_row[d]) * v_scale;
+          }
+        }
+        for (int32_t h = j * G; h < (j + 1) * G; ++h) {
+          const uint16_t* q_row = q + t * q_stride_t + (int64_t)h * q_stride_h;
+          float* out_row = out + (r * Hq + h) * (int64_t)D;
+          for (int32_t d = 0; d < D; ++d) out_row[d] = 0.0f;
+          if (n == 0) continue; /* fully masked row or zero width: exactly zero */
+          /* 3. scores */
+          for (int64_t i = 0; i < n; ++i) {
+            float acc = 0.0f;
+            for (int32_t d = 0; d < D; ++d) acc += bf16_to_float(q_row[d]) * kf[i * D + d];
+            sc[i] = scale * acc;
+          }
+          /* 4. softmax over the selected slots */
+          float m = sc[0];
+          for (int64_t i = 1; i < n; ++i)
+            if (sc[i] > m) m = sc[i];
+          float l = 0.0f;
+          for (int64_t i = 0; i < n; ++i) {
+            sc[i] = expf(sc[i] - m);
+            l += sc[i];
+          }
+          /* 5. P V, normalised */
+          for (int64_t i = 0; i < n; ++i)
+            for (int32_t d = 0; d < D; ++d) out_row[d] += sc[i] * vf[i * D + d];
+          for (int32_t d = 0; d < D; ++d) out_row[d] = out_row[d] / l;
+        }
+      }
+    }
+    free(sel);
+    free(kf);
+    free(vf);
+    free(sc);
+    all_bits |= bits;
+  }
+  if (err_bits) *err_bits |= all_bits;
+  return 0;
+}
+
 /* Number of OpenMP threads a parallel region of this library uses (1 without OpenMP). */
 int qsa_oracle_num_threads(void) {
 #ifdef _OPENMP

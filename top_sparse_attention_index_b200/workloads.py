@@ -41,6 +41,9 @@ class Workload:
     scales: tuple = (DEFAULT_SCALE,)
     notes: dict = field(default_factory=dict)
     block: int = 1              # slots named by one entry of slot_idx (block selection)
+    kv_format: str = "bf16"     # "bf16", or "e4m3": k_cache / v_cache hold float8_e4m3fn codes
+    k_scale: float = 1.0        # dequantisation scales of an e4m3 cache
+    v_scale: float = 1.0
 
     @property
     def Tq(self) -> int:
@@ -241,6 +244,38 @@ def max_extent(Hq: int = 6, clustered: bool = False, seed: int | None = None) ->
         idx = _shuffle_rows(gen, torch.cat([window, outside], dim=1)).to(torch.int32)
     return Workload("max_extent_hq%d_hkv1_s262144_tq4096_w2048_%s" % (Hq, "clustered" if clustered else "uniform"),
                     q, k, v, idx, None)
+
+
+# --------------------------------------------------------------------------------------
+# fp8_e4m3 KV cache ("Where this sits in the Qwen4Exp serving build-out": fp8_e4m3 is the
+# KV-cache format that performed better for this attention's decode).
+# --------------------------------------------------------------------------------------
+
+# Per-tensor scales for N(0,1) data: |x| / scale stays below the largest finite E4M3
+# magnitude (448) for |x| < 6, and the smallest |x| land in the subnormal codes.
+E4M3_K_SCALE = 0.0135
+E4M3_V_SCALE = 0.0125
+
+
+def to_e4m3_cache(x: torch.Tensor, scale: float) -> torch.Tensor:
+    """float8_e4m3fn codes of x / scale (round to nearest, clamped to +-448): how a KV
+    writer stores a cache with one scale per tensor."""
+    return (x.float() / scale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+
+
+def with_e4m3_cache(w: Workload, k_scale: float = E4M3_K_SCALE,
+                    v_scale: float = E4M3_V_SCALE) -> Workload:
+    """The same workload with its K and V caches stored as E4M3 codes."""
+    return Workload(w.name + "_e4m3kv", w.q, to_e4m3_cache(w.k_cache, k_scale),
+                    to_e4m3_cache(w.v_cache, v_scale), w.slot_idx, w.width, scales=w.scales,
+                    notes=dict(w.notes), block=w.block, kv_format="e4m3", k_scale=k_scale,
+                    v_scale=v_scale)
+
+
+def long_prefill_e4m3kv(seed: int = 1238) -> Workload:
+    """The long-prefill case with an fp8_e4m3 K/V cache (the bf16 case's values, scaled
+    by 1/0.0135 for K and 1/0.0125 for V and rounded to E4M3)."""
+    return with_e4m3_cache(long_prefill(seed))
 
 
 CONFIGS = {

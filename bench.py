@@ -40,6 +40,7 @@ METRIC = "sparse prefill TFLOP/s & query-slot pairs/s, 7810q×2051 sel; % of roo
 WORKLOADS = {
     "long_prefill": lambda: wl.long_prefill(),
     "long_prefill_block4": lambda: wl.long_prefill_block4(),
+    "long_prefill_e4m3kv": lambda: wl.long_prefill_e4m3kv(),
     "tiny": lambda: wl.tiny(),
     "width_sweep": lambda: wl.width_sweep(),
     "causal_two_request": lambda: wl.causal_two_request(),
@@ -87,7 +88,8 @@ def work_counts(w: wl.Workload):
     pairs = int(pairs_per_row(w).sum())
     D = w.q.shape[2]
     flops = pairs * w.Hq * 4 * D                         # 2D (QK^T) + 2D (PV) per head
-    gathered = pairs * w.Hkv * 2 * D * 2                 # K and V rows, bf16 (pairs count slots)
+    kv_bytes = 1 if w.kv_format == "e4m3" else 2
+    gathered = pairs * w.Hkv * 2 * D * kv_bytes          # K and V rows (pairs count slots)
     other = w.Tq * w.Hq * D * 2 * 2 + w.Tq * W * 4       # Q in, out, indices
     return pairs, flops, gathered + other, gathered
 
@@ -179,13 +181,22 @@ def cpu_baseline(w: wl.Workload, target_s: float):
     o = oracle.default()
     scale = w.scales[0]
     probe = list(range(min(16, w.Tq)))
+
+    def fwd(rows):
+        if w.kv_format == "e4m3":
+            o.forward_fp8kv(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, w.k_scale,
+                            w.v_scale, rows=rows, block=w.block)
+        else:
+            o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=rows,
+                      block=w.block)
+
     t0 = time.perf_counter()
-    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=probe, block=w.block)
+    fwd(probe)
     dt = max(time.perf_counter() - t0, 1e-3)
     n = int(min(w.Tq, max(64, len(probe) * target_s / dt)))
     rows = list(range(n))
     t0 = time.perf_counter()
-    o.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, scale, rows=rows, block=w.block)
+    fwd(rows)
     dt = time.perf_counter() - t0
     flops = int(pairs_per_row(w)[:n].sum()) * w.Hq * 4 * 256
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": o.num_threads(),
@@ -255,7 +266,8 @@ def main():
     if args.rows:
         w = wl.Workload(f"{w.name}_rows{args.rows}", w.q[:args.rows], w.k_cache, w.v_cache,
                         w.slot_idx[:args.rows], None if w.width is None else w.width[:args.rows],
-                        scales=w.scales, block=w.block)
+                        scales=w.scales, block=w.block, kv_format=w.kv_format,
+                        k_scale=w.k_scale, v_scale=w.v_scale)
     pairs, flops, alg_bytes, gathered = work_counts(w)
     q, k, v, idx = (x.to(device) for x in (w.q, w.k_cache, w.v_cache, w.slot_idx))
     width = None if w.width is None else w.width.to(device)
@@ -269,7 +281,8 @@ def main():
     stream = torch.cuda.current_stream(device)
 
     def step():
-        qsa.sparse_prefill(q, k, v, idx, width, scale=scale, out=out, block=w.block)
+        qsa.sparse_prefill(q, k, v, idx, width, scale=scale, out=out, block=w.block,
+                           k_scale=w.k_scale, v_scale=w.v_scale)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -319,7 +332,8 @@ def main():
 
         def e2e_step():
             _, fin = qsa.sparse_prefill_from_host(hq, hk, hv, hidx, w.width, scale=scale,
-                                                  out=hout, device=device, block=w.block)
+                                                  out=hout, device=device, block=w.block,
+                                                  k_scale=w.k_scale, v_scale=w.v_scale)
             return fin
 
         for _ in range(3):
@@ -360,7 +374,8 @@ def main():
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        # the MMA input type (bf16 caches: bf16; E4M3 caches: f16 from the 8-bit codes)
+        "dtype": "f16 (e4m3 kv)" if w.kv_format == "e4m3" else "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": 256, "S": w.S,
                    "W": w.W, "valid_pairs": pairs, "nsplit": nsplit,

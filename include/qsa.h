@@ -63,6 +63,9 @@ typedef enum {
 /* Bits that the kernels OR into *err_word (device memory, optional). */
 #define QSA_ERRBIT_SLOT_RANGE 0x1u /* a slot index outside [-1, S) was seen; it was masked */
 #define QSA_ERRBIT_WIDTH_RANGE 0x2u /* a width[t] outside [0, W] was seen; it was clamped   */
+#define QSA_ERRBIT_Q_RANGE 0x4u     /* fp8-KV entry point only: a query element with
+                                       |q| >= 65536 (beyond the f16 range the fp8-KV
+                                       products run in); that row's output is not valid  */
 
 /* Largest number of selected positions one split processes (the per-split index list
  * is staged whole in shared memory).  Wider selections are split automatically. */
@@ -160,6 +163,45 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
                                       int32_t D, int64_t S, int32_t W, int32_t block, float scale,
                                       void* out, int64_t out_stride_t, int64_t out_stride_h,
                                       int32_t nsplit, void* workspace, size_t workspace_bytes,
+                                      uint32_t* err_word, void* stream);
+
+/*
+ * qsa_sparse_prefill_fp8kv -- the same attention over an fp8_e4m3 K/V cache.
+ *
+ * Source: the article "Qwen4-Exp QSA comes to Huawei's Ascend: inside SGLang's opt-in
+ * CANN prefill PR", section "Where this sits in the Qwen4Exp serving build-out", which
+ * reports fp8_e4m3 as the KV-cache format that performed better for this attention's
+ * decode.  Reading taken here: k_cache and v_cache hold one OCP FP8 E4M3 code per
+ * element (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals, NaN =
+ * S.1111.111, no infinities) and each tensor carries one float scale, so the
+ * dequantised element is value(code) * k_scale (resp. v_scale).  What one call
+ * computes is the definition at the top of this file with
+ *   k_cache[s, j, d] := value(k_code[s, j, d]) * k_scale,
+ *   v_cache[s, j, d] := value(v_code[s, j, d]) * v_scale.
+ * Dequantisation happens on the gathered rows inside the kernel; the cache is read-only.
+ *
+ * Arguments are those of qsa_sparse_prefill_block, except:
+ *   k_cache, v_cache   E4M3 codes (one byte each) [S, Hkv, D]; strides
+ *                      (k_stride_s, k_stride_h, 1) in elements = bytes, each a
+ *                      non-negative multiple of 16; base 16-byte aligned.
+ *   k_scale, v_scale   finite floats (QSA_ERR_INVALID_ARG otherwise).
+ * q and out stay bf16 with the alignment rules of qsa_sparse_prefill.  The split plan
+ * and workspace are those of qsa_sparse_prefill_block_plan for the same shape and
+ * block.  Numerics: the products run on f16 tensor-core inputs with fp32 accumulation;
+ * every E4M3 value is exact in f16 and a bf16 query element is exact in f16 for
+ * 2^-17 <= |q| < 65536 (smaller magnitudes lose low bits, at most 2^-25 absolute);
+ * a query element with |q| >= 65536 sets QSA_ERRBIT_Q_RANGE and its row's output is
+ * not valid.  Code NaN in the cache propagates as NaN.
+ */
+qsa_status_t qsa_sparse_prefill_fp8kv(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                      const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                      const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                      const int32_t* slot_idx, int64_t idx_stride_t,
+                                      const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                      int32_t D, int64_t S, int32_t W, int32_t block, float scale,
+                                      float k_scale, float v_scale, void* out,
+                                      int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
+                                      void* workspace, size_t workspace_bytes,
                                       uint32_t* err_word, void* stream);
 
 /* Size of the device scratch array that qsa_sparse_prefill_noalloc uses (16 MiB). */

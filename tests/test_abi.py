@@ -178,3 +178,54 @@ def test_wrapper_refuses_cpu_tensors():
     idx = torch.zeros(2, 3, dtype=torch.int32)
     with pytest.raises(ValueError):
         qsa.sparse_prefill(q, k, k, idx)
+
+
+def _call8(**over):
+    """A raw call of the fp8_e4m3-KV entry point with fake aligned pointers (strides of
+    the E4M3 caches in bytes); each case makes one argument invalid."""
+    a = dict(q=0x10000, q_stride_t=16 * 256, q_stride_h=256, k_cache=0x20000, k_stride_s=512,
+             k_stride_h=256, v_cache=0x30000, v_stride_s=512, v_stride_h=256, slot_idx=0x40000,
+             idx_stride_t=8, width=None, Tq=4, Hq=16, Hkv=2, D=256, S=100, W=8, block=1,
+             scale=0.0625, k_scale=0.0135, v_scale=0.0125, out=0x50000, out_stride_t=16 * 256,
+             out_stride_h=256, nsplit=1, workspace=None, workspace_bytes=0, err_word=None,
+             stream=None)
+    a.update(over)
+    return qsa.qsa_sparse_prefill_fp8kv(**a)
+
+
+INVALID8 = [
+    (dict(k_stride_h=264), qsa.QSA_ERR_INVALID_ARG),    # 264 bytes: not a multiple of 16
+    (dict(v_stride_s=520), qsa.QSA_ERR_INVALID_ARG),
+    (dict(k_cache=0x20008), qsa.QSA_ERR_INVALID_ARG),   # misaligned base
+    (dict(k_scale=float("nan")), qsa.QSA_ERR_INVALID_ARG),
+    (dict(v_scale=float("inf")), qsa.QSA_ERR_INVALID_ARG),
+    (dict(block=0), qsa.QSA_ERR_INVALID_ARG),
+    (dict(q_stride_h=260), qsa.QSA_ERR_INVALID_ARG),     # q stays bf16: multiples of 8
+    (dict(D=128), qsa.QSA_ERR_UNSUPPORTED),
+    (dict(k_stride_s=2 ** 32), qsa.QSA_ERR_UNSUPPORTED),  # slot stride of 4 GiB
+    (dict(nsplit=2, workspace=None), qsa.QSA_ERR_WORKSPACE),
+]
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="fake-pointer validation runs only where no GPU can be reached")
+@pytest.mark.parametrize("over,status", INVALID8, ids=[str(o) for o, _ in INVALID8])
+def test_fp8kv_invalid_arguments_rejected_before_launch(lib, over, status):
+    assert _call8(**over) == status
+    assert qsa.qsa_last_error_detail() != ""
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_fp8kv_strides_accepted_up_to_the_device_query(lib):
+    # E4M3 strides are bytes: any multiple of 16 is accepted; with valid arguments the
+    # automatic split reaches the device query, which fails without a GPU
+    assert _call8(k_stride_h=272, nsplit=0) == qsa.QSA_ERR_CUDA
+    assert _call8(Tq=0, q=None, k_cache=None, v_cache=None, out=None, slot_idx=None) == qsa.QSA_OK
+
+
+def test_wrapper_refuses_cpu_fp8_tensors():
+    q = torch.zeros(2, 16, 256, dtype=torch.bfloat16)
+    k = torch.zeros(4, 2, 256, dtype=torch.float8_e4m3fn)
+    idx = torch.zeros(2, 3, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        qsa.sparse_prefill(q, k, k, idx, k_scale=0.5, v_scale=0.5)

@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     QSA_ERR_UNSUPPORTED,
     QSA_ERR_WORKSPACE,
     QSA_ERRBIT_SLOT_RANGE,
+    QSA_ERRBIT_Q_RANGE,
     QSA_ERRBIT_WIDTH_RANGE,
     QSA_MAX_BLOCK,
     QSA_MAX_SLOTS_PER_SPLIT,
@@ -23,6 +24,7 @@ from ._binding import (  # noqa: F401
     qsa_sparse_prefill,
     qsa_sparse_prefill_block,
     qsa_sparse_prefill_block_plan,
+    qsa_sparse_prefill_fp8kv,
     qsa_sparse_prefill_noalloc,
     qsa_sparse_prefill_plan,
     qsa_status_string,
@@ -32,7 +34,7 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "sparse_prefill", "sparse_prefill_from_host", "qsa_sparse_prefill", "qsa_sparse_prefill_noalloc",
-    "qsa_sparse_prefill_block", "qsa_sparse_prefill_block_plan",
+    "qsa_sparse_prefill_block", "qsa_sparse_prefill_block_plan", "qsa_sparse_prefill_fp8kv",
     "qsa_sparse_prefill_plan", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
     "load_library", "QSAError",
 ]

@@ -21,6 +21,7 @@ QSA_ERR_WORKSPACE = 3
 QSA_ERR_CUDA = 4
 QSA_ERRBIT_SLOT_RANGE = 0x1
 QSA_ERRBIT_WIDTH_RANGE = 0x2
+QSA_ERRBIT_Q_RANGE = 0x4
 QSA_MAX_SLOTS_PER_SPLIT = 2240
 QSA_MAX_BLOCK = 16
 QSA_STATIC_SCRATCH_BYTES = 16 << 20
@@ -38,6 +39,9 @@ SIGNATURES = {
     "qsa_sparse_prefill_block": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64,
                                         _p, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _f, _p, _i64,
                                         _i64, _i32, _p, _sz, _p, _p]),
+    "qsa_sparse_prefill_fp8kv": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64,
+                                        _p, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _f, _f, _f,
+                                        _p, _i64, _i64, _i32, _p, _sz, _p, _p]),
     "qsa_sparse_prefill_noalloc": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _f, _p,
                                           _i64, _i64, _i32, _p, _p]),
@@ -131,6 +135,19 @@ def qsa_sparse_prefill_block(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_s
         workspace_bytes, err_word, stream))
 
 
+def qsa_sparse_prefill_fp8kv(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,
+                             v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv,
+                             D, S, W, block, scale, k_scale, v_scale, out, out_stride_t,
+                             out_stride_h, nsplit, workspace, workspace_bytes, err_word,
+                             stream) -> int:
+    """Raw call with an E4M3 K/V cache (strides in bytes) and its two scales."""
+    return int(load_library().qsa_sparse_prefill_fp8kv(
+        q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache, v_stride_s,
+        v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W, block,
+        ctypes.c_float(scale), ctypes.c_float(k_scale), ctypes.c_float(v_scale), out,
+        out_stride_t, out_stride_h, nsplit, workspace, workspace_bytes, err_word, stream))
+
+
 def qsa_sparse_prefill_noalloc(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
                                v_cache, v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq,
                                Hq, Hkv, D, S, W, scale, out, out_stride_t, out_stride_h, nsplit,
@@ -159,14 +176,16 @@ def _check_dev(name, t, dtype, device):
 
 
 def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=None, nsplit=0,
-                   err_word=None, stream=None, block=1):
+                   err_word=None, stream=None, block=1, k_scale=1.0, v_scale=1.0):
     """Selected-slot sparse attention on the GPU.
 
     q [Tq, Hq, 256] bf16, k_cache / v_cache [S, Hkv, 256] bf16, slot_idx [Tq, W] int32
     (-1 = masked), width [Tq] int32 or None; scale defaults to 1/sqrt(256) = 1/16.
     Returns out [Tq, Hq, 256] bf16 (allocated unless given).  Work is enqueued on
     ``stream`` (default: torch's current stream); nothing is synchronised.  With
-    block > 1 every entry of slot_idx names `block` consecutive slots.
+    block > 1 every entry of slot_idx names `block` consecutive slots.  K/V caches of
+    dtype float8_e4m3fn are an fp8_e4m3 cache dequantised as code value x k_scale
+    (x v_scale); the scales are ignored for bf16 caches.
     """
     device = q.device
     if device.type != "cuda":
@@ -178,8 +197,10 @@ def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=No
     if slot_idx.dim() != 2 or slot_idx.shape[0] != Tq:
         raise ValueError("slot_idx must be [Tq, W]")
     W = slot_idx.shape[1]
-    for name, t, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, torch.bfloat16),
-                        ("v_cache", v_cache, torch.bfloat16), ("slot_idx", slot_idx, torch.int32)):
+    kv_fp8 = k_cache.dtype == torch.float8_e4m3fn
+    kv_dt = torch.float8_e4m3fn if kv_fp8 else torch.bfloat16
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, kv_dt),
+                        ("v_cache", v_cache, kv_dt), ("slot_idx", slot_idx, torch.int32)):
         _check_dev(name, t, dt, device)
     if width is not None:
         _check_dev("width", width, torch.int32, device)
@@ -199,11 +220,15 @@ def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=No
     ns, ws_bytes = qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, block, num_sms, nsplit)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device) if ws_bytes else None
     with torch.cuda.device(device):
-        st = qsa_sparse_prefill_block(
-            _ptr(q), q.stride(0), q.stride(1), _ptr(k_cache), k_cache.stride(0), k_cache.stride(1),
-            _ptr(v_cache), v_cache.stride(0), v_cache.stride(1), _ptr(slot_idx) if W else None,
-            slot_idx.stride(0), _ptr(width), Tq, Hq, Hkv, D, S, W, block, float(scale), _ptr(out),
-            out.stride(0), out.stride(1), ns, _ptr(ws), ws_bytes, _ptr(err_word), stream.cuda_stream)
+        head = (_ptr(q), q.stride(0), q.stride(1), _ptr(k_cache), k_cache.stride(0), k_cache.stride(1),
+                _ptr(v_cache), v_cache.stride(0), v_cache.stride(1), _ptr(slot_idx) if W else None,
+                slot_idx.stride(0), _ptr(width), Tq, Hq, Hkv, D, S, W, block, float(scale))
+        tail = (_ptr(out), out.stride(0), out.stride(1), ns, _ptr(ws), ws_bytes, _ptr(err_word),
+                stream.cuda_stream)
+        if kv_fp8:
+            st = qsa_sparse_prefill_fp8kv(*head, float(k_scale), float(v_scale), *tail)
+        else:
+            st = qsa_sparse_prefill_block(*head, *tail)
     if st != QSA_OK:
         raise QSAError(st, qsa_last_error_detail())
     return out
@@ -223,7 +248,8 @@ def _copy_streams(device):
 
 
 def sparse_prefill_from_host(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=None,
-                             device=None, chunk_rows=None, nsplit=0, block=1):
+                             device=None, chunk_rows=None, nsplit=0, block=1, k_scale=1.0,
+                             v_scale=1.0):
     """Host-buffer form of sparse_prefill: copies the inputs to `device`, runs the kernels
     and copies the result back, overlapping the transfers with the computation.
 
@@ -276,7 +302,7 @@ def sparse_prefill_from_host(q, k_cache, v_cache, slot_idx, width=None, scale=No
                 if t is not None:
                     t.record_stream(comp)
             sparse_prefill(q_c, k_d, v_d, i_c, w_c, scale=scale, out=out_d[r0:r1], nsplit=nsplit,
-                           stream=comp, block=block)
+                           stream=comp, block=block, k_scale=k_scale, v_scale=v_scale)
             done = torch.cuda.Event()
             done.record(comp)
             d2h.wait_event(done)

@@ -149,15 +149,22 @@ int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, 
                                        workspace_bytes);
 }
 
-qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t q_stride_h,
-                                      const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
-                                      const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
-                                      const int32_t* slot_idx, int64_t idx_stride_t,
-                                      const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
-                                      int32_t D, int64_t S, int32_t W, int32_t block, float scale,
-                                      void* out, int64_t out_stride_t, int64_t out_stride_h,
-                                      int32_t nsplit, void* workspace, size_t workspace_bytes,
-                                      uint32_t* err_word, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The body shared by every launching entry point.  kv_fp8: k_cache / v_cache hold E4M3
+// codes (one byte per element, strides multiples of 16) dequantised with k_scale and
+// v_scale; otherwise bf16 (strides multiples of 8 elements) and the scales are 1.
+qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                          const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                          const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                          const int32_t* slot_idx, int64_t idx_stride_t, const int32_t* width,
+                          int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int64_t S, int32_t W,
+                          int32_t block, float scale, bool kv_fp8, float k_scale, float v_scale,
+                          void* out, int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
+                          void* workspace, size_t workspace_bytes, uint32_t* err_word,
+                          void* stream) {
   g_detail[0] = '\0';
   qsa_status_t st = check_shape(Tq, Hq, Hkv, D, W);
   if (st == QSA_OK) st = check_block(block);
@@ -165,6 +172,8 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
   if (S < 0) return fail(QSA_ERR_INVALID_ARG, "negative S");
   if (nsplit < 0) return fail(QSA_ERR_INVALID_ARG, "negative nsplit");
   if (!std::isfinite(scale)) return fail(QSA_ERR_INVALID_ARG, "scale is not finite");
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return fail(QSA_ERR_INVALID_ARG, "k_scale or v_scale is not finite");
   if (Tq == 0) return QSA_OK;
 
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr)
@@ -175,13 +184,19 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
   if ((slot_idx != nullptr && !aligned4(slot_idx)) || (width != nullptr && !aligned4(width)) ||
       (err_word != nullptr && !aligned4(err_word)))
     return fail(QSA_ERR_INVALID_ARG, "slot_idx, width and err_word must be 4-byte aligned");
-  if (!stride_ok(q_stride_t) || !stride_ok(q_stride_h) || !stride_ok(k_stride_s) ||
-      !stride_ok(k_stride_h) || !stride_ok(v_stride_s) || !stride_ok(v_stride_h) ||
-      !stride_ok(out_stride_t) || !stride_ok(out_stride_h))
-    return fail(QSA_ERR_INVALID_ARG, "tensor strides must be non-negative multiples of 8 elements");
+  if (!stride_ok(q_stride_t) || !stride_ok(q_stride_h) || !stride_ok(out_stride_t) ||
+      !stride_ok(out_stride_h))
+    return fail(QSA_ERR_INVALID_ARG, "q and out strides must be non-negative multiples of 8 elements");
+  // K / V strides: 16 bytes = 8 bf16 elements or 16 E4M3 codes.
+  const int64_t kv_elem = kv_fp8 ? 1 : 2;
+  const auto kv_stride_ok = [&](int64_t x) { return x >= 0 && (x * kv_elem) % 16 == 0; };
+  if (!kv_stride_ok(k_stride_s) || !kv_stride_ok(k_stride_h) || !kv_stride_ok(v_stride_s) ||
+      !kv_stride_ok(v_stride_h))
+    return fail(QSA_ERR_INVALID_ARG, "k_cache / v_cache strides must be non-negative multiples of %d elements",
+                int(16 / kv_elem));
   if (idx_stride_t < 0) return fail(QSA_ERR_INVALID_ARG, "negative idx_stride_t");
   // The kernels step from slot to slot by a 32-bit byte stride.
-  if (uint64_t(k_stride_s) * 2 > UINT32_MAX || uint64_t(v_stride_s) * 2 > UINT32_MAX)
+  if (uint64_t(k_stride_s) * kv_elem > UINT32_MAX || uint64_t(v_stride_s) * kv_elem > UINT32_MAX)
     return fail(QSA_ERR_UNSUPPORTED, "slot stride of 4 GiB or more");
 
   int32_t num_sms = 0;
@@ -204,8 +219,8 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
 
   qsa::FwdParams p{};
   p.q = static_cast<const uint16_t*>(q);
-  p.k_cache = static_cast<const uint16_t*>(k_cache);
-  p.v_cache = static_cast<const uint16_t*>(v_cache);
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
   p.slot_idx = slot_idx;
   p.width = width;
   p.out = static_cast<uint16_t*>(out);
@@ -232,14 +247,52 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
   p.W = W;
   p.nsplit = pl.nsplit;
   p.split_len = pl.split_len;
-  p.k_row_bytes = uint32_t(k_stride_s * 2);
-  p.v_row_bytes = uint32_t(v_stride_s * 2);
-  p.scale_log2 = scale * 1.4426950408889634f;  // log2(e): the kernels use 2^x
+  p.k_row_bytes = uint32_t(k_stride_s * kv_elem);
+  p.v_row_bytes = uint32_t(v_stride_s * kv_elem);
+  // log2(e): the kernels use 2^x; an E4M3 cache's k_scale multiplies every score
+  p.scale_log2 = kv_fp8 ? scale * k_scale * 1.4426950408889634f : scale * 1.4426950408889634f;
   p.block = block;
+  p.kv_fp8 = kv_fp8 ? 1 : 0;
+  p.v_scale = kv_fp8 ? v_scale : 1.0f;
 
   const cudaError_t e = qsa::launch_sparse_prefill(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
   return QSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                      const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                      const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                      const int32_t* slot_idx, int64_t idx_stride_t,
+                                      const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                      int32_t D, int64_t S, int32_t W, int32_t block, float scale,
+                                      void* out, int64_t out_stride_t, int64_t out_stride_h,
+                                      int32_t nsplit, void* workspace, size_t workspace_bytes,
+                                      uint32_t* err_word, void* stream) {
+  return prefill_impl(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,
+                      v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W,
+                      block, scale, false, 1.0f, 1.0f, out, out_stride_t, out_stride_h, nsplit,
+                      workspace, workspace_bytes, err_word, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_fp8kv(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                      const void* k_cache, int64_t k_stride_s, int64_t k_stride_h,
+                                      const void* v_cache, int64_t v_stride_s, int64_t v_stride_h,
+                                      const int32_t* slot_idx, int64_t idx_stride_t,
+                                      const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                      int32_t D, int64_t S, int32_t W, int32_t block, float scale,
+                                      float k_scale, float v_scale, void* out,
+                                      int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
+                                      void* workspace, size_t workspace_bytes,
+                                      uint32_t* err_word, void* stream) {
+  return prefill_impl(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,
+                      v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W,
+                      block, scale, true, k_scale, v_scale, out, out_stride_t, out_stride_h, nsplit,
+                      workspace, workspace_bytes, err_word, stream);
 }
 
 qsa_status_t qsa_sparse_prefill(const void* q, int64_t q_stride_t, int64_t q_stride_h,

@@ -45,13 +45,14 @@ constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent)
 
 
-template <int NTILE, int DSPLIT, int SL, int STAGES>
+template <int NTILE, int DSPLIT, int SL, int STAGES, bool KV8 = false>
 struct Cfg {
   static constexpr int kParts = NTILE * DSPLIT;  // warps serving one slot lane
   static constexpr int kWarps = kParts * SL;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kRows = 16 * SL;                      // slots per stage
-  static constexpr int kSubBytes = 16 * kRowBytes * 2;       // one sub-tile: 16 K rows, 16 V rows
+  static constexpr int kKvRow = KV8 ? kHeadDim : kRowBytes;  // one gathered K or V row (bytes)
+  static constexpr int kSubBytes = 16 * kKvRow * 2;          // one sub-tile: 16 K rows, 16 V rows
   static constexpr int kStageBytes = SL * kSubBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;    // [slot lane][stage][sub-tile]
   static constexpr int kQBytes = NTILE * 8 * kRowBytes;
@@ -72,13 +73,20 @@ struct Cfg {
 // NTILE n8 tiles cover the head group (G <= 8: 1; G <= 16: 2).  The warps of one slot
 // lane split either the head tiles (NTILE = 2) or, with DSPLIT = 2, the D rows of the PV
 // product (both compute the same scores).
-template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT>
+// KV8: the cache holds E4M3 codes (256-byte rows).  The gathered codes stay 8-bit in
+// shared memory and become f16 in registers right after ldmatrix (cvt.f16x2.e4m3x2, exact);
+// Q and P are f16 too, so both products are f16 MMAs with fp32 accumulation.  The order
+// of the D index inside a k-step (Q K^T) or an m-tile (P V) is permuted to match what
+// ldmatrix delivers for 8-bit data; a sum over D does not depend on that order, and the
+// epilogue maps the m-tile rows back.
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8>
 __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p) {
   static_assert(NTILE == 1 || DSPLIT == 1, "a lane splits either the heads or D");
   static_assert(!QSPLIT || DSPLIT == 2, "splitting Q K^T needs a D-split pair");
   constexpr int kKS = QSPLIT ? 8 : 16;  // k-steps of Q K^T per warp
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8>;
+  constexpr int kKvRow = C::kKvRow;
   constexpr int kMT = 16 / DSPLIT;  // m16 tiles of D per warp in the PV product
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
@@ -203,34 +211,61 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
   // chunk offsets (row & 7 is a compile-time
   // constant in the unrolled loop because a lane's rows start at 0 or 8), so a
   // destination is a register plus an immediate.
+  // An E4M3 row is 16 chunks: lanes 0-15 copy one row, lanes 16-31 the next.
+  constexpr int kElem = KV8 ? 1 : 2;
+  const uint32_t lchunk = KV8 ? uint32_t(lane & 15) : uint32_t(lane);
+  const int lhalf = KV8 ? (lane >> 4) : 0;
   const uint64_t kg = static_cast<uint64_t>(__cvta_generic_to_global(
-                          p.k_cache + int64_t(j) * p.k_stride_h)) + uint64_t(lane) * 16;
+                          static_cast<const uint8_t*>(p.k_cache) + int64_t(j) * p.k_stride_h * kElem)) +
+                      uint64_t(lchunk) * 16;
   const uint64_t vg = static_cast<uint64_t>(__cvta_generic_to_global(
-                          p.v_cache + int64_t(j) * p.v_stride_h)) + uint64_t(lane) * 16;
+                          static_cast<const uint8_t*>(p.v_cache) + int64_t(j) * p.v_stride_h * kElem)) +
+                      uint64_t(lchunk) * 16;
   const uint32_t kstride = p.k_row_bytes, vstride = p.v_row_bytes;
-  const uint32_t lane16 = uint32_t(lane) << 4;
+  const uint32_t lane16 = lchunk << 4;
   // this lane's sub-tiles: [wslot][stage]; a warp pair splits the 16 rows 8 / 8
   const uint32_t sub_s = ring_s + wslot * STAGES * C::kSubBytes;
   constexpr int kLoadRows = 16 / C::kParts;
   const int row0 = wpart * kLoadRows;
-  const uint32_t sub_rows = sub_s + row0 * kRowBytes;
+  const uint32_t sub_rows = sub_s + (row0 + lhalf) * kKvRow;
 
   auto load_stage = [&](int s, int buf) {
     const int base = s * C::kRows + wslot * 16;
     if (base >= n_valid) return;  // an empty sub-tile is neither loaded nor read
-    uint32_t kd[8];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (m << 4));
     const uint4* slots = reinterpret_cast<const uint4*>(sSlot + base + row0);  // 16-byte aligned
+    if constexpr (!KV8) {
+      uint32_t kd[8];
 #pragma unroll
-    for (int i = 0; i < kLoadRows; i += 4) {
-      const uint4 s4 = slots[i / 4];  // slots of rows i .. i + 3
-      const uint32_t sl[4] = {s4.x, s4.y, s4.z, s4.w};
+      for (int m = 0; m < 8; ++m) kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (m << 4));
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t d = kd[(i + e) & 7] + (i + e) * kRowBytes;
-        cp_async_16_global(d, kg + uint64_t(sl[e]) * kstride);
-        cp_async_16_global(d + 16 * kRowBytes, vg + uint64_t(sl[e]) * vstride);
+      for (int i = 0; i < kLoadRows; i += 4) {
+        const uint4 s4 = slots[i / 4];  // slots of rows i .. i + 3
+        const uint32_t sl[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t d = kd[(i + e) & 7] + (i + e) * kRowBytes;
+          cp_async_16_global(d, kg + uint64_t(sl[e]) * kstride);
+          cp_async_16_global(d + 16 * kRowBytes, vg + uint64_t(sl[e]) * vstride);
+        }
+      }
+    } else {
+      // instruction ip copies rows 2 ip + lhalf; their swizzle key is (2 ip + lhalf) & 7
+      uint32_t kd[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (uint32_t((2 * m + lhalf) & 7) << 4));
+#pragma unroll
+      for (int i = 0; i < kLoadRows; i += 4) {
+        const uint4 s4 = slots[i / 4];  // slots of rows i .. i + 3
+        const uint32_t sa = lhalf ? s4.y : s4.x;  // row i + lhalf
+        const uint32_t sb = lhalf ? s4.w : s4.z;  // row i + 2 + lhalf
+        const int ip = i / 2;
+        uint32_t d = kd[ip & 3] + ip * 2 * kKvRow;
+        cp_async_16_global(d, kg + uint64_t(sa) * kstride);
+        cp_async_16_global(d + 16 * kKvRow, vg + uint64_t(sa) * vstride);
+        d = kd[(ip + 1) & 3] + (ip + 1) * 2 * kKvRow;
+        cp_async_16_global(d, kg + uint64_t(sb) * kstride);
+        cp_async_16_global(d + 16 * kKvRow, vg + uint64_t(sb) * vstride);
       }
     }
   };
@@ -256,16 +291,36 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
   // (with QSPLIT, warp wd of a pair keeps the k-steps of its half of D only)
   uint32_t qf[kKS][2];
   const int ks0 = QSPLIT ? wd * kKS : 0;
+  if constexpr (!KV8) {
 #pragma unroll
-  for (int kp = 0; kp < kKS / 2; ++kp) {
-    const int g = lane & 7;
-    const int c = 4 * kp + 2 * ks0 + (lane >> 3);
-    uint32_t r[4];
-    ldmatrix_x4(r, q_s + (wn * 8 + g) * kRowBytes + ((c ^ g) << 4));
-    qf[2 * kp][0] = r[0];
-    qf[2 * kp][1] = r[1];
-    qf[2 * kp + 1][0] = r[2];
-    qf[2 * kp + 1][1] = r[3];
+    for (int kp = 0; kp < kKS / 2; ++kp) {
+      const int g = lane & 7;
+      const int c = 4 * kp + 2 * ks0 + (lane >> 3);
+      uint32_t r[4];
+      ldmatrix_x4(r, q_s + (wn * 8 + g) * kRowBytes + ((c ^ g) << 4));
+      qf[2 * kp][0] = r[0];
+      qf[2 * kp][1] = r[1];
+      qf[2 * kp + 1][0] = r[2];
+      qf[2 * kp + 1][1] = r[3];
+    }
+  } else {
+    // f16 B fragments in the permuted k order of the E4M3 A fragments: for k-step ks
+    // (D range 16 ks .. 16 ks + 15) lane l holds head l/4, elements 16 ks + 4 (l%4) + 0..3.
+    const int n = wn * 8 + (lane >> 2);
+    bool q_big = false;
+#pragma unroll
+    for (int ks = 0; ks < kKS; ++ks) {
+      const int c8 = 2 * (ks0 + ks) + ((lane & 3) >> 1);
+      const uint2 v = *reinterpret_cast<const uint2*>(sQ + n * kRowBytes + ((c8 ^ (n & 7)) << 4) +
+                                                      8 * (lane & 1));
+      const float f0 = bf16lo_to_f32(v.x), f1 = bf16hi_to_f32(v.x);
+      const float f2 = bf16lo_to_f32(v.y), f3 = bf16hi_to_f32(v.y);
+      q_big |= fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))) >= 65536.f;
+      qf[ks][0] = pack_f16x2(f0, f1);
+      qf[ks][1] = pack_f16x2(f2, f3);
+    }
+    if (__any_sync(0xffffffffu, q_big) && lane == 0 && p.err_word != nullptr)
+      atomicOr(p.err_word, 4u);
   }
 
   // ---- 3. main loop ------------------------------------------------------------------
@@ -288,8 +343,10 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
   uint32_t kswz[4], vswz[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    kswz[m] = uint32_t(krow * kRowBytes + (((2 * m + khi) ^ key) << 4));
-    vswz[m] = uint32_t(16 * kRowBytes + vrow * kRowBytes + (((2 * m + vhi) ^ key) << 4));
+    kswz[m] = uint32_t(krow * kKvRow + (((2 * m + khi) ^ key) << 4));
+    // E4M3 V: the transposed loads use the K lane pattern (one chunk is one m-tile)
+    vswz[m] = KV8 ? kswz[m] + 16 * kKvRow
+                  : uint32_t(16 * kRowBytes + vrow * kRowBytes + (((2 * m + vhi) ^ key) << 4));
   }
   const float sl2 = p.scale_log2;
 
@@ -309,15 +366,31 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8); two chains for ILP.
     uint32_t kt[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) kt[m] = sub + kswz[m] + ks0 * 32;  // 16 k-steps = 4 x 128 B
+    for (int m = 0; m < 4; ++m) kt[m] = sub + kswz[m] + ks0 * (KV8 ? 16 : 32);  // a k-step's bytes
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (!KV8) {
 #pragma unroll
-    for (int ks = 0; ks < kKS; ks += 2) {
-      uint32_t a[4];
-      ldmatrix_x4(a, kt[ks & 3] + 128 * (ks >> 2));
-      mma_bf16_16816(sa, a, qf[ks][0], qf[ks][1]);
-      ldmatrix_x4(a, kt[(ks + 1) & 3] + 128 * ((ks + 1) >> 2));
-      mma_bf16_16816(sb, a, qf[ks + 1][0], qf[ks + 1][1]);
+      for (int ks = 0; ks < kKS; ks += 2) {
+        uint32_t a[4];
+        ldmatrix_x4(a, kt[ks & 3] + 128 * (ks >> 2));
+        mma_bf16_16816(sa, a, qf[ks][0], qf[ks][1]);
+        ldmatrix_x4(a, kt[(ks + 1) & 3] + 128 * ((ks + 1) >> 2));
+        mma_bf16_16816(sb, a, qf[ks + 1][0], qf[ks + 1][1]);
+      }
+    } else {
+      // one ldmatrix.x4 = two k-steps of 8-bit codes: r0 / r1 = rows 0-7 / 8-15 of
+      // chunk 2 kq, r2 / r3 of chunk 2 kq + 1; lane l holds 4 codes of row l/4
+#pragma unroll
+      for (int kq = 0; kq < kKS / 2; ++kq) {
+        uint32_t r[4], a[4];
+        ldmatrix_x4(r, kt[kq & 3] + 128 * (kq >> 2));
+        e4m3x4_to_f16x2x2(r[0], a[0], a[2]);
+        e4m3x4_to_f16x2x2(r[1], a[1], a[3]);
+        mma_f16_16816(sa, a, qf[2 * kq][0], qf[2 * kq][1]);
+        e4m3x4_to_f16x2x2(r[2], a[0], a[2]);
+        e4m3x4_to_f16x2x2(r[3], a[1], a[3]);
+        mma_f16_16816(sb, a, qf[2 * kq + 1][0], qf[2 * kq + 1][1]);
+      }
     }
     float s0 = sa[0] + sb[0], s1 = sa[1] + sb[1], s2 = sa[2] + sb[2], s3 = sa[3] + sb[3];
     if constexpr (QSPLIT) {
@@ -372,23 +445,52 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
       m0 = mn0;
       m1 = mn1;
     }
-    const uint32_t p01 = pack_bf16x2(fast_exp2(x0 - m0), fast_exp2(x1 - m1));
-    const uint32_t p23 = pack_bf16x2(fast_exp2(x2 - m0), fast_exp2(x3 - m1));
-    // the denominators sum the same bf16-rounded weights that multiply V
-    l0 += bf16lo_to_f32(p01) + bf16lo_to_f32(p23);
-    l1 += bf16hi_to_f32(p01) + bf16hi_to_f32(p23);
+    uint32_t p01, p23;
+    if constexpr (!KV8) {
+      p01 = pack_bf16x2(fast_exp2(x0 - m0), fast_exp2(x1 - m1));
+      p23 = pack_bf16x2(fast_exp2(x2 - m0), fast_exp2(x3 - m1));
+      // the denominators sum the same bf16-rounded weights that multiply V
+      l0 += bf16lo_to_f32(p01) + bf16lo_to_f32(p23);
+      l1 += bf16hi_to_f32(p01) + bf16hi_to_f32(p23);
+    } else {
+      // f16 weights (<= 2^kRescaleLog2, in range) for the f16 P V product
+      p01 = pack_f16x2(fast_exp2(x0 - m0), fast_exp2(x1 - m1));
+      p23 = pack_f16x2(fast_exp2(x2 - m0), fast_exp2(x3 - m1));
+      l0 += f16lo_to_f32(p01) + f16lo_to_f32(p23);
+      l1 += f16hi_to_f32(p01) + f16hi_to_f32(p23);
+    }
 
     // O^T (this warp's D rows x 8) += V^T (D rows x 16) * P^T (16 x 8)
     const uint32_t b0 = movmatrix_trans(p01);
     const uint32_t b1 = movmatrix_trans(p23);
     uint32_t vt[4];
+    if constexpr (!KV8) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / 4) * 128;
+      for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / 4) * 128;
 #pragma unroll
-    for (int mt = 0; mt < kMT; ++mt) {
-      uint32_t a[4];
-      ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
-      mma_bf16_16816(o[mt], a, b0, b1);
+      for (int mt = 0; mt < kMT; ++mt) {
+        uint32_t a[4];
+        ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
+        mma_bf16_16816(o[mt], a, b0, b1);
+      }
+    } else {
+      // m-tile = one 16-byte chunk of D.  Transposed 8-bit loads give lane l the codes
+      // (slot 2(l%4) and 2(l%4)+1) x (d = 16 c + 2(l/4) and + 1); a byte permute pairs
+      // the two slots of each d, so tile row l/4 is d = 16 c + 2(l/4) and row l/4 + 8
+      // is d + 1.  r0 / r1: slots 0-7 / 8-15 of chunk 2 mq, r2 / r3 of chunk 2 mq + 1.
+#pragma unroll
+      for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / 8) * 128;
+#pragma unroll
+      for (int mq = 0; mq < kMT / 2; ++mq) {
+        uint32_t r[4], a[4];
+        ldmatrix_x4_trans(r, vt[mq & 3] + 128 * (mq >> 2));
+        e4m3x4_to_f16x2x2(byte_perm(r[0], 0u, 0x3120u), a[0], a[1]);
+        e4m3x4_to_f16x2x2(byte_perm(r[1], 0u, 0x3120u), a[2], a[3]);
+        mma_f16_16816(o[2 * mq], a, b0, b1);
+        e4m3x4_to_f16x2x2(byte_perm(r[2], 0u, 0x3120u), a[0], a[1]);
+        e4m3x4_to_f16x2x2(byte_perm(r[3], 0u, 0x3120u), a[2], a[3]);
+        mma_f16_16816(o[2 * mq + 1], a, b0, b1);
+      }
     }
   }
   cp_async_wait<0>();
@@ -408,11 +510,14 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     const int r8 = lane >> 2;
 #pragma unroll
     for (int mt = 0; mt < kMT; ++mt) {
-      const int d = 16 * (wd * kMT + mt) + r8;
+      // rows r8 / r8 + 8 of the m-tile are d = 16 mt' + r8 / + 8 (bf16), or
+      // d = 16 mt' + 2 r8 / + 1 (E4M3 order)
+      constexpr int kHi = KV8 ? 1 : 8;
+      const int d = 16 * (wd * kMT + mt) + (KV8 ? 2 * r8 : r8);
       mine[g0 * kMergeStride + d] = o[mt][0];
       mine[(g0 + 1) * kMergeStride + d] = o[mt][1];
-      mine[g0 * kMergeStride + d + 8] = o[mt][2];
-      mine[(g0 + 1) * kMergeStride + d + 8] = o[mt][3];
+      mine[g0 * kMergeStride + d + kHi] = o[mt][2];
+      mine[(g0 + 1) * kMergeStride + d + kHi] = o[mt][3];
     }
     if (r8 == 0) {
       mine[8 * kMergeStride + g0] = m0;
@@ -448,7 +553,7 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
       acc[0] += sc * a.x; acc[1] += sc * a.y; acc[2] += sc * a.z; acc[3] += sc * a.w;
       acc[4] += sc * b.x; acc[5] += sc * b.y; acc[6] += sc * b.z; acc[7] += sc * b.w;
     }
-    const float inv = 1.f / lsum;
+    const float inv = (KV8 ? p.v_scale : 1.f) / lsum;
     const int64_t h = head0 + gg;
     if (p.nsplit == 1) {
       uint4 v;
@@ -504,10 +609,10 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
   *dst = v;
 }
 
-template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT>
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES>;
-  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8>;
+  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8>;
   // The shared-memory opt-in is a per-device function attribute: set it on the first
   // launch on each device only, so later calls (e.g. under stream capture) are launches
   // and nothing else.
@@ -555,10 +660,27 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
 #ifndef QSA_SMALL_QSPLIT
 #define QSA_SMALL_QSPLIT true
 #endif
+// E4M3 caches: a sub-tile is half the bytes, so each slot lane runs a deeper pipeline.
+#ifndef QSA_FP8_SMALL_SL
+#define QSA_FP8_SMALL_SL 3
+#endif
+#ifndef QSA_FP8_SMALL_STAGES
+#define QSA_FP8_SMALL_STAGES 4
+#endif
+#ifndef QSA_FP8_LARGE_SL
+#define QSA_FP8_LARGE_SL 3
+#endif
+#ifndef QSA_FP8_LARGE_STAGES
+#define QSA_FP8_LARGE_STAGES 3
+#endif
 using CfgSmall = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES>;
 using CfgLarge = Cfg<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES>;
+using CfgSmall8 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true>;
+using CfgLarge8 = Cfg<2, 1, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, true>;
 static_assert(CfgSmall::kSmem <= CfgSmall::kSmPerCta(QSA_SMALL_CTAS), "small shape: CTAs per SM");
 static_assert(CfgLarge::kSmem <= CfgLarge::kSmPerCta(QSA_LARGE_CTAS), "large shape: CTAs per SM");
+static_assert(CfgSmall8::kSmem <= CfgSmall8::kSmPerCta(QSA_SMALL_CTAS), "E4M3 small shape: CTAs per SM");
+static_assert(CfgLarge8::kSmem <= CfgLarge8::kSmPerCta(QSA_LARGE_CTAS), "E4M3 large shape: CTAs per SM");
 
 }  // namespace
 
@@ -582,11 +704,18 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
 }
 
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
-  cudaError_t e = (p.G <= 8)
-                      ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES,
-                                   QSA_SMALL_CTAS, QSA_SMALL_QSPLIT>(p, stream)
-                      : launch_fwd<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS, false>(
-                            p, stream);
+  cudaError_t e;
+  if (p.kv_fp8) {
+    e = (p.G <= 8) ? launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
+                                true>(p, stream)
+                   : launch_fwd<2, 1, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, QSA_LARGE_CTAS, false,
+                                true>(p, stream);
+  } else {
+    e = (p.G <= 8) ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
+                                QSA_SMALL_QSPLIT, false>(p, stream)
+                   : launch_fwd<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS, false, false>(
+                         p, stream);
+  }
   if (e != cudaSuccess || p.nsplit == 1) return e;
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);

@@ -21,8 +21,8 @@ constexpr int kMaxBlock = 16;           // largest block size of block selection
 // Everything one launch of the fused kernel needs (passed by value).
 struct FwdParams {
   const uint16_t* q;        // bf16 bits [Tq, Hq, D]
-  const uint16_t* k_cache;  // bf16 bits [S, Hkv, D]
-  const uint16_t* v_cache;
+  const void* k_cache;      // [S, Hkv, D]: bf16 bits, or E4M3 codes when kv_fp8
+  const void* v_cache;
   const int32_t* slot_idx;  // [Tq, W] row stride idx_stride_t
   const int32_t* width;     // [Tq] or nullptr
   uint16_t* out;            // bf16 bits [Tq, Hq, D]
@@ -38,10 +38,12 @@ struct FwdParams {
   int32_t Tq, Hq, Hkv, G, W;
   int32_t nsplit;
   int32_t split_len;        // positions of the W axis per split
-  uint32_t k_row_bytes;     // k_stride_s * 2: one slot step of K in bytes
-  uint32_t v_row_bytes;     // v_stride_s * 2
-  float scale_log2;         // scale * log2(e)
+  uint32_t k_row_bytes;     // k_stride_s * element bytes: one slot step of K in bytes
+  uint32_t v_row_bytes;     // v_stride_s * element bytes
+  float scale_log2;         // scale * log2(e) (times k_scale for an E4M3 cache)
   int32_t block;            // slots named by one selected entry (1 = slot selection)
+  int32_t kv_fp8;           // 1: k_cache / v_cache hold E4M3 codes
+  float v_scale;            // E4M3 cache: multiplier of the normalised output
 };
 
 // Kernel configuration chosen for a group size G (shared by planner and launcher).

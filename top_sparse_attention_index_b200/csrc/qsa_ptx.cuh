@@ -2,8 +2,9 @@
 //
 // Asynchronous global->shared copies (cp.async, 16 bytes, zero-fill when the source
 // size is 0), warp-wide 8x8 matrix loads from shared memory (ldmatrix), the bf16
-// m16n8k16 warp MMA with fp32 accumulation, the in-register 8x8 transpose (movmatrix)
-// and the base-2 exponent / logarithm instructions.
+// and f16 m16n8k16 warp MMAs with fp32 accumulation, the in-register 8x8 transpose
+// (movmatrix), E4M3 -> f16 conversion, byte permutes and the base-2 exponent /
+// logarithm instructions.
 #pragma once
 
 #include <cstdint>
@@ -62,6 +63,54 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D = A(16x16, row) * B(16x8, col) + D, f16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Four E4M3 codes (bytes 0..3 of x) -> two packed f16x2: `lo` holds bytes 0 and 1 (byte 0
+// in the low half), `hi` bytes 2 and 3.  Exact: every E4M3 value is an f16 value.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{\n"
+      "  .reg .b16 a, b;\n"
+      "  mov.b32 {a, b}, %2;\n"
+      "  cvt.rn.f16x2.e4m3x2 %0, a;\n"
+      "  cvt.rn.f16x2.e4m3x2 %1, b;\n"
+      "}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+// Byte permute: result byte i = byte (sel >> 4i) & 7 of the pair {y:x} (x = bytes 0..3).
+__device__ __forceinline__ uint32_t byte_perm(uint32_t x, uint32_t y, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(r) : "r"(x), "r"(y), "r"(sel));
+  return r;
+}
+
+// Two floats -> packed f16x2 (round to nearest even); `lo` lands in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float f16lo_to_f32(uint32_t x) {
+  float f;
+  asm("{\n  .reg .b16 a, b;\n  mov.b32 {a, b}, %1;\n  cvt.f32.f16 %0, a;\n}\n" : "=f"(f) : "r"(x));
+  return f;
+}
+__device__ __forceinline__ float f16hi_to_f32(uint32_t x) {
+  float f;
+  asm("{\n  .reg .b16 a, b;\n  mov.b32 {a, b}, %1;\n  cvt.f32.f16 %0, b;\n}\n" : "=f"(f) : "r"(x));
+  return f;
 }
 
 // Transpose of an 8x8 b16 matrix held in the standard fragment layout (lane l owns

@@ -360,9 +360,11 @@ def main():
     traffic = None
     prof = ROOT / "profiles" / "traffic.json"
     if prof.exists():
-        tj = json.loads(prof.read_text())
-        if tj.get("kernel_source_hash") == _kernel_hash() and tj.get("workload_name") == w.name:
-            traffic = tj.get("bytes_per_launch")
+        # one record per workload; a record counts only while the kernel sources it was
+        # captured with are unchanged
+        for rec in json.loads(prof.read_text()).get("records", []):
+            if rec.get("kernel_source_hash") == _kernel_hash() and rec.get("workload_name") == w.name:
+                traffic = rec.get("bytes_per_launch")
     result = {
         "metric": METRIC,
         "value": world * flops / t_s / 1e12,

@@ -27,6 +27,13 @@
 //      (exact zeros for empty rows), or fp32 partials + base-2 LSE when split.
 // K2 qsa_lse_combine_kernel -- one warp per (t, h): log-sum-exp weighted sum of the
 //   split partials; empty splits carry LSE = -inf and weight 0; all empty -> exact 0.
+//
+// fp8_e4m3 KV cache (the format named in section "Where this sits in the Qwen4Exp serving
+// build-out" of the same article): K1 with KV8 gathers 256-byte rows of E4M3 codes (half
+// the bytes), keeps them 8-bit in shared memory and converts them to f16 in registers
+// after ldmatrix; Q, P and both MMAs are f16 with fp32 accumulation; k_scale is folded
+// into the softmax scale and v_scale into the final normalisation, so the result is the
+// attention over the dequantised cache up to rounding.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -660,12 +667,14 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
 #ifndef QSA_SMALL_QSPLIT
 #define QSA_SMALL_QSPLIT true
 #endif
-// E4M3 caches: a sub-tile is half the bytes, so each slot lane runs a deeper pipeline.
+// E4M3 caches: a sub-tile is half the bytes, so the same shared memory holds more slot
+// lanes (G <= 8: four lanes of three stages, 16 warps per SM, measured best) or a deeper
+// pipeline per lane.
 #ifndef QSA_FP8_SMALL_SL
-#define QSA_FP8_SMALL_SL 3
+#define QSA_FP8_SMALL_SL 4
 #endif
 #ifndef QSA_FP8_SMALL_STAGES
-#define QSA_FP8_SMALL_STAGES 4
+#define QSA_FP8_SMALL_STAGES 3
 #endif
 #ifndef QSA_FP8_LARGE_SL
 #define QSA_FP8_LARGE_SL 3

@@ -173,6 +173,15 @@ def test_forced_splits_decode_shape(cuda_device, oracle_lib, nsplit):
     check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"nsplit={nsplit}")
 
 
+def test_head_major_order_four_kv_heads(cuda_device, oracle_lib):
+    """A 128 MB cache of four 32 MB head slices: the launch orders its work units KV head
+    slowest (the long prefill does too, with two heads); every head's rows must land."""
+    w = _random_case(79, 300, 16, 4, 32768, 700, minus1=0.05, widths=True)
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    rows = list(range(0, w.Tq, 3)) + [w.Tq - 1]
+    compare_rows(w, got, oracle_lib, 1.0 / 16.0, rows, "4 KV heads, head-major")
+
+
 def test_rows_wider_than_one_split(cuda_device, oracle_lib):
     """W = 6,000 > 2,240 slots per split forces at least three splits."""
     w = _random_case(78, 300, 16, 2, 20000, 6000, minus1=0.1, widths=True)

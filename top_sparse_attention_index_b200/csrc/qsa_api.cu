@@ -254,6 +254,7 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
   p.block = block;
   p.kv_fp8 = kv_fp8 ? 1 : 0;
   p.v_scale = kv_fp8 ? v_scale : 1.0f;
+  p.head_major = qsa::kernel_order_head_major(S, Hkv, int32_t(kv_elem));
 
   const cudaError_t e = qsa::launch_sparse_prefill(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));

@@ -113,11 +113,14 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
                                            // Q K^T with QSPLIT)
 
   // ---- work unit -------------------------------------------------------------------
+  // head_major: KV head slowest, so the CTAs resident at any time gather from one head's
+  // slice of the cache (S rows per tensor) instead of all Hkv heads'; otherwise the
+  // heads of a query row are neighbours and share its index row in L2.
   int u = blockIdx.x;
   const int split = u % p.nsplit;
   u /= p.nsplit;
-  const int j = u % p.Hkv;
-  const int t = u / p.Hkv;
+  const int j = p.head_major ? u / p.Tq : u % p.Hkv;
+  const int t = p.head_major ? u % p.Tq : u / p.Hkv;
 
   int width_t = p.W;
   if (p.width != nullptr) {

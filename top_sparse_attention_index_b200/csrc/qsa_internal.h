@@ -44,6 +44,7 @@ struct FwdParams {
   int32_t block;            // slots named by one selected entry (1 = slot selection)
   int32_t kv_fp8;           // 1: k_cache / v_cache hold E4M3 codes
   float v_scale;            // E4M3 cache: multiplier of the normalised output
+  int32_t head_major;       // 1: work units ordered KV head slowest (see kernel_order)
 };
 
 // Kernel configuration chosen for a group size G (shared by planner and launcher).
@@ -58,6 +59,16 @@ struct KernelShape {
 };
 
 KernelShape kernel_shape(int G);
+
+// Work-unit order of K1: KV head slowest when the whole K/V cache is larger than
+// kHeadMajorBytes (about three quarters of B200's 126 MB L2) and one head's slice is
+// smaller, so the resident CTAs keep one L2-sized slice hot; otherwise the heads of a
+// query row run side by side and share its index row.
+constexpr double kHeadMajorBytes = 96.0 * 1024 * 1024;
+inline int32_t kernel_order_head_major(int64_t S, int32_t Hkv, int32_t kv_elem_bytes) {
+  const double slice = double(S) * kHeadDim * kv_elem_bytes * 2;  // one head's K and V
+  return (Hkv > 1 && slice * Hkv > kHeadMajorBytes && slice <= kHeadMajorBytes) ? 1 : 0;
+}
 
 // Enqueue the fused kernel (and the combine when nsplit > 1) on `stream`.
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream);

@@ -390,6 +390,9 @@ def main():
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": alg_bytes},
+        # the bound that binds once the gathered rows are L2 hits: every gathered byte
+        # is written to shared memory once (cp.async) and read once (ldmatrix)
+        "shared_memory": _smem_bound(gathered, t_s, clocks.summary(t0_epoch, t1_epoch)),
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks.summary(t0_epoch, t1_epoch),
         "wall_s_timed_region": t_wall,
@@ -399,6 +402,16 @@ def main():
     if not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(result))
+
+
+def _smem_bound(gathered: int, t_s: float, clk: dict, sms: int = 148) -> dict:
+    """Shared-memory round-trip roofline: 2 x gathered bytes against sms x 128 B per
+    SM clock at the median SM clock sampled during the timed region."""
+    mhz = clk.get("sm_mhz") or 1965.0
+    peak = sms * 128 * mhz * 1e6 / 1e12
+    achieved = 2 * gathered / t_s / 1e12
+    return {"bytes_per_launch": 2 * gathered, "achieved": achieved, "peak": peak,
+            "unit": "TB/s", "frac": achieved / peak, "sm_mhz": mhz}
 
 
 def _kernel_hash():

@@ -54,7 +54,10 @@ constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent
 
 template <int NTILE, int DSPLIT, int SL, int STAGES, bool KV8 = false>
 struct Cfg {
-  static constexpr int kParts = NTILE * DSPLIT;  // warps serving one slot lane
+  // warps serving one slot lane: a D-split pair (each warp handles every head tile over
+  // its half of D) or one warp per head tile
+  static constexpr int kParts = DSPLIT > 1 ? DSPLIT : NTILE;
+  static constexpr int kTPW = DSPLIT > 1 ? NTILE : 1;  // head tiles per warp
   static constexpr int kWarps = kParts * SL;
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kRows = 16 * SL;                      // slots per stage
@@ -66,11 +69,18 @@ struct Cfg {
   static constexpr int kIdxBytes = kMaxSlotsPerSplit * 4;  // compacted slot numbers
   static constexpr int kScanBytes = 32 * 4;
   // partial scores a D-split pair exchanges when it also splits Q K^T: [lane][warp][32][4]
-  static constexpr int kXchgBytes = (DSPLIT > 1) ? SL * DSPLIT * 32 * 16 : 0;
-  static constexpr int kMergeBytes = kWarps * (8 * kMergeStride + 16) * 4;
+  static constexpr int kXchgBytes = (DSPLIT > 1) ? SL * DSPLIT * kTPW * 32 * 16 : 0;
+  static constexpr int kTileFloats = 8 * kMergeStride + 16;  // one head tile's merge record
+  static constexpr int kMergeBytes = kWarps * kTPW * kTileFloats * 4;
+  // with two head tiles per warp the exchange buffer overlays the Q tile, which is dead
+  // once the Q fragments are in registers
+  static constexpr bool kXchgOverQ = kTPW > 1;
+  static_assert(!kXchgOverQ || kXchgBytes <= kQBytes, "exchange buffer fits the Q tile");
   static constexpr size_t kSmem =
-      size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes + kXchgBytes;
-  static_assert(kMergeBytes <= kRingBytes, "merge buffer reuses the ring");
+      size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes + (kXchgOverQ ? 0 : kXchgBytes);
+  // the epilogue's merge buffer reuses the ring and, after it, the Q tile and the slot
+  // list (all dead once the main loop is over)
+  static_assert(kMergeBytes <= kRingBytes + kQBytes + kIdxBytes, "merge buffer fits");
   static_assert(kMaxSlotsPerSplit * 4 <= kRingBytes, "raw index staging reuses the ring");
   static_assert(kMaxSlotsPerSplit % 16 == 0, "the offset list pads to whole sub-tiles");
   // shared memory one SM gives its resident CTAs (228 KiB, 1 KiB reserved per CTA)
@@ -78,8 +88,10 @@ struct Cfg {
 };
 
 // NTILE n8 tiles cover the head group (G <= 8: 1; G <= 16: 2).  The warps of one slot
-// lane split either the head tiles (NTILE = 2) or, with DSPLIT = 2, the D rows of the PV
-// product (both compute the same scores).
+// lane split either the head tiles (DSPLIT = 1: one warp per tile) or, with DSPLIT = 2,
+// the D rows of the PV product, each warp handling every head tile (and with QSPLIT also
+// the D range of Q K^T, the pair exchanging partial scores), so every gathered row is
+// read from shared memory once.
 // KV8: the cache holds E4M3 codes (256-byte rows).  The gathered codes stay 8-bit in
 // shared memory and become f16 in registers right after ldmatrix (cvt.f16x2.e4m3x2, exact);
 // Q and P are f16 too, so both products are f16 MMAs with fp32 accumulation.  The order
@@ -87,28 +99,29 @@ struct Cfg {
 // ldmatrix delivers for 8-bit data; a sum over D does not depend on that order, and the
 // epilogue maps the m-tile rows back.
 template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8>
-__global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
+__global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p) {
-  static_assert(NTILE == 1 || DSPLIT == 1, "a lane splits either the heads or D");
   static_assert(!QSPLIT || DSPLIT == 2, "splitting Q K^T needs a D-split pair");
   constexpr int kKS = QSPLIT ? 8 : 16;  // k-steps of Q K^T per warp
   using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8>;
   constexpr int kKvRow = C::kKvRow;
   constexpr int kMT = 16 / DSPLIT;  // m16 tiles of D per warp in the PV product
+  constexpr int TPW = C::kTPW;      // n8 head tiles per warp
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ring = smem;
   uint8_t* sQ = smem + C::kRingBytes;
   // Compacted valid slot numbers of the split, padded to whole 16-slot sub-tiles.
   uint32_t* sSlot = reinterpret_cast<uint32_t*>(sQ + C::kQBytes);
   int32_t* sScan = reinterpret_cast<int32_t*>(sSlot + kMaxSlotsPerSplit);
-  float4* sXchg = reinterpret_cast<float4*>(sScan + 32);  // (DSPLIT > 1 and QSPLIT only)
+  float4* sXchg = C::kXchgOverQ ? reinterpret_cast<float4*>(sQ)  // (QSPLIT only)
+                                 : reinterpret_cast<float4*>(sScan + 32);
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int wslot = warp % SL;  // which 16-slot sub-tile of a stage
   const int wpart = warp / SL;             // which warp of the slot lane
-  const int wn = NTILE > 1 ? wpart : 0;    // which n8 tile of the head group
+  const int wn = DSPLIT == 1 ? wpart : 0;  // first n8 tile of this warp
   const int wd = DSPLIT > 1 ? wpart : 0;   // which D range of the PV product (and of
                                            // Q K^T with QSPLIT)
 
@@ -299,46 +312,59 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
 
   // B fragments of Q^T for this warp's n8 tile, all 16 k-steps of D = 256.
   // (with QSPLIT, warp wd of a pair keeps the k-steps of its half of D only)
-  uint32_t qf[kKS][2];
+  uint32_t qf[TPW][kKS][2];
   const int ks0 = QSPLIT ? wd * kKS : 0;
   if constexpr (!KV8) {
 #pragma unroll
-    for (int kp = 0; kp < kKS / 2; ++kp) {
-      const int g = lane & 7;
-      const int c = 4 * kp + 2 * ks0 + (lane >> 3);
-      uint32_t r[4];
-      ldmatrix_x4(r, q_s + (wn * 8 + g) * kRowBytes + ((c ^ g) << 4));
-      qf[2 * kp][0] = r[0];
-      qf[2 * kp][1] = r[1];
-      qf[2 * kp + 1][0] = r[2];
-      qf[2 * kp + 1][1] = r[3];
+    for (int nt = 0; nt < TPW; ++nt) {
+#pragma unroll
+      for (int kp = 0; kp < kKS / 2; ++kp) {
+        const int g = lane & 7;
+        const int c = 4 * kp + 2 * ks0 + (lane >> 3);
+        uint32_t r[4];
+        ldmatrix_x4(r, q_s + ((wn + nt) * 8 + g) * kRowBytes + ((c ^ g) << 4));
+        qf[nt][2 * kp][0] = r[0];
+        qf[nt][2 * kp][1] = r[1];
+        qf[nt][2 * kp + 1][0] = r[2];
+        qf[nt][2 * kp + 1][1] = r[3];
+      }
     }
   } else {
     // f16 B fragments in the permuted k order of the E4M3 A fragments: for k-step ks
     // (D range 16 ks .. 16 ks + 15) lane l holds head l/4, elements 16 ks + 4 (l%4) + 0..3.
-    const int n = wn * 8 + (lane >> 2);
     bool q_big = false;
 #pragma unroll
-    for (int ks = 0; ks < kKS; ++ks) {
-      const int c8 = 2 * (ks0 + ks) + ((lane & 3) >> 1);
-      const uint2 v = *reinterpret_cast<const uint2*>(sQ + n * kRowBytes + ((c8 ^ (n & 7)) << 4) +
-                                                      8 * (lane & 1));
-      const float f0 = bf16lo_to_f32(v.x), f1 = bf16hi_to_f32(v.x);
-      const float f2 = bf16lo_to_f32(v.y), f3 = bf16hi_to_f32(v.y);
-      q_big |= fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))) >= 65536.f;
-      qf[ks][0] = pack_f16x2(f0, f1);
-      qf[ks][1] = pack_f16x2(f2, f3);
+    for (int nt = 0; nt < TPW; ++nt) {
+      const int n = (wn + nt) * 8 + (lane >> 2);
+#pragma unroll
+      for (int ks = 0; ks < kKS; ++ks) {
+        const int c8 = 2 * (ks0 + ks) + ((lane & 3) >> 1);
+        const uint2 v = *reinterpret_cast<const uint2*>(sQ + n * kRowBytes +
+                                                        ((c8 ^ (n & 7)) << 4) + 8 * (lane & 1));
+        const float f0 = bf16lo_to_f32(v.x), f1 = bf16hi_to_f32(v.x);
+        const float f2 = bf16lo_to_f32(v.y), f3 = bf16hi_to_f32(v.y);
+        q_big |= fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))) >= 65536.f;
+        qf[nt][ks][0] = pack_f16x2(f0, f1);
+        qf[nt][ks][1] = pack_f16x2(f2, f3);
+      }
     }
     if (__any_sync(0xffffffffu, q_big) && lane == 0 && p.err_word != nullptr)
       atomicOr(p.err_word, 4u);
   }
+  if constexpr (C::kXchgOverQ) __syncthreads();  // Q fragments loaded: the exchange may reuse sQ
 
   // ---- 3. main loop ------------------------------------------------------------------
-  float m0 = kNegInf, m1 = kNegInf;  // reference max (base 2) of heads 2(l%4), 2(l%4)+1
-  float l0 = 0.f, l1 = 0.f;          // this lane's share of the running sums
-  float o[kMT][4];
+  // per head tile nt of this warp: reference max (base 2) and this lane's share of the
+  // running sums of heads 2(l%4), 2(l%4)+1, and the O^T accumulators
+  float m0[TPW], m1[TPW], l0[TPW], l1[TPW];
+  float o[TPW][kMT][4];
 #pragma unroll
-  for (int mt = 0; mt < kMT; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  for (int nt = 0; nt < TPW; ++nt) {
+    m0[nt] = m1[nt] = kNegInf;
+    l0[nt] = l1[nt] = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+  }
 
   // ldmatrix addressing.  Chunk c of a row sits at ((c ^ key) << 4), key = row & 7 =
   // lane & 7 for every row this lane addresses.  With c = 2 * step + hi (step = k-step
@@ -373,19 +399,27 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     if (base >= n_valid) continue;  // warp-uniform: no valid slot in this sub-tile
     const uint32_t sub = sub_s + buf * C::kSubBytes;
 
-    // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8); two chains for ILP.
+    // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8) per head tile; each K
+    // fragment feeds every tile of the warp; two chains for ILP.
     uint32_t kt[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) kt[m] = sub + kswz[m] + ks0 * (KV8 ? 16 : 32);  // a k-step's bytes
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    float sa[TPW][4], sb[TPW][4];
+#pragma unroll
+    for (int nt = 0; nt < TPW; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sa[nt][e] = sb[nt][e] = 0.f;
     if constexpr (!KV8) {
 #pragma unroll
       for (int ks = 0; ks < kKS; ks += 2) {
         uint32_t a[4];
         ldmatrix_x4(a, kt[ks & 3] + 128 * (ks >> 2));
-        mma_bf16_16816(sa, a, qf[ks][0], qf[ks][1]);
+#pragma unroll
+        for (int nt = 0; nt < TPW; ++nt) mma_bf16_16816(sa[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
         ldmatrix_x4(a, kt[(ks + 1) & 3] + 128 * ((ks + 1) >> 2));
-        mma_bf16_16816(sb, a, qf[ks + 1][0], qf[ks + 1][1]);
+#pragma unroll
+        for (int nt = 0; nt < TPW; ++nt)
+          mma_bf16_16816(sb[nt], a, qf[nt][ks + 1][0], qf[nt][ks + 1][1]);
       }
     } else {
       // one ldmatrix.x4 = two k-steps of 8-bit codes: r0 / r1 = rows 0-7 / 8-15 of
@@ -396,33 +430,52 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
         ldmatrix_x4(r, kt[kq & 3] + 128 * (kq >> 2));
         e4m3x4_to_f16x2x2(r[0], a[0], a[2]);
         e4m3x4_to_f16x2x2(r[1], a[1], a[3]);
-        mma_f16_16816(sa, a, qf[2 * kq][0], qf[2 * kq][1]);
+#pragma unroll
+        for (int nt = 0; nt < TPW; ++nt)
+          mma_f16_16816(sa[nt], a, qf[nt][2 * kq][0], qf[nt][2 * kq][1]);
         e4m3x4_to_f16x2x2(r[2], a[0], a[2]);
         e4m3x4_to_f16x2x2(r[3], a[1], a[3]);
-        mma_f16_16816(sb, a, qf[2 * kq + 1][0], qf[2 * kq + 1][1]);
+#pragma unroll
+        for (int nt = 0; nt < TPW; ++nt)
+          mma_f16_16816(sb[nt], a, qf[nt][2 * kq + 1][0], qf[nt][2 * kq + 1][1]);
       }
     }
-    float s0 = sa[0] + sb[0], s1 = sa[1] + sb[1], s2 = sa[2] + sb[2], s3 = sa[3] + sb[3];
+    float sc[TPW][4];
+#pragma unroll
+    for (int nt = 0; nt < TPW; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = sa[nt][e] + sb[nt][e];
     if constexpr (QSPLIT) {
       // each warp of the pair holds the scores over its half of D: exchange and add in
       // a fixed order (low half + high half) so both warps hold the same scores
-      float4* mine = sXchg + (wslot * 2 + wd) * 32 + lane;
-      float4* other = sXchg + (wslot * 2 + (wd ^ 1)) * 32 + lane;
-      *mine = make_float4(s0, s1, s2, s3);
+#pragma unroll
+      for (int nt = 0; nt < TPW; ++nt)
+        sXchg[((wslot * 2 + wd) * TPW + nt) * 32 + lane] =
+            make_float4(sc[nt][0], sc[nt][1], sc[nt][2], sc[nt][3]);
       named_barrier_sync(1 + wslot, 64);
-      const float4 t = *other;
-      if (wd == 0) {
-        s0 += t.x; s1 += t.y; s2 += t.z; s3 += t.w;
-      } else {
-        s0 = t.x + s0; s1 = t.y + s1; s2 = t.z + s2; s3 = t.w + s3;
+#pragma unroll
+      for (int nt = 0; nt < TPW; ++nt) {
+        const float4 t = sXchg[((wslot * 2 + (wd ^ 1)) * TPW + nt) * 32 + lane];
+        if (wd == 0) {
+          sc[nt][0] += t.x; sc[nt][1] += t.y; sc[nt][2] += t.z; sc[nt][3] += t.w;
+        } else {
+          sc[nt][0] = t.x + sc[nt][0]; sc[nt][1] = t.y + sc[nt][1];
+          sc[nt][2] = t.z + sc[nt][2]; sc[nt][3] = t.w + sc[nt][3];
+        }
       }
     }
-    float x0 = s0 * sl2, x1 = s1 * sl2;
-    float x2 = s2 * sl2, x3 = s3 * sl2;
+    float x[TPW][4];
+#pragma unroll
+    for (int nt = 0; nt < TPW; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[nt][e] = sc[nt][e] * sl2;
     if (base + 16 > n_valid) {  // warp-uniform: only the last sub-tile has padding rows
       const int r0 = base + (lane >> 2);
-      if (r0 >= n_valid) x0 = x1 = kNegInf;
-      if (r0 + 8 >= n_valid) x2 = x3 = kNegInf;
+#pragma unroll
+      for (int nt = 0; nt < TPW; ++nt) {
+        if (r0 >= n_valid) x[nt][0] = x[nt][1] = kNegInf;
+        if (r0 + 8 >= n_valid) x[nt][2] = x[nt][3] = kNegInf;
+      }
     }
 
     // Online softmax over the slot axis (rows); lanes sharing l%4 hold one head pair.
@@ -432,47 +485,60 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     // is unchanged.  A vote on the lanes' own maxima decides whether any head moves;
     // only then is the exact chunk max reduced over the slot axis (the decision is the
     // same as comparing the exact max).  The max is finite: row `base` is valid.
-    const float lx0 = fmaxf(x0, x2), lx1 = fmaxf(x1, x3);
-    if (__any_sync(0xffffffffu, lx0 > m0 + kRescaleLog2 || lx1 > m1 + kRescaleLog2)) {
-      float mx0 = lx0, mx1 = lx1;
+    bool need = false;
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const float mn0 = (mx0 > m0 + kRescaleLog2) ? mx0 : m0;
-      const float mn1 = (mx1 > m1 + kRescaleLog2) ? mx1 : m1;
-      const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);  // -inf -> 0
-      l0 *= al0;
-      l1 *= al1;
+    for (int nt = 0; nt < TPW; ++nt)
+      need |= fmaxf(x[nt][0], x[nt][2]) > m0[nt] + kRescaleLog2 ||
+              fmaxf(x[nt][1], x[nt][3]) > m1[nt] + kRescaleLog2;
+    if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-      for (int mt = 0; mt < kMT; ++mt) {
-        o[mt][0] *= al0;
-        o[mt][1] *= al1;
-        o[mt][2] *= al0;
-        o[mt][3] *= al1;
+      for (int nt = 0; nt < TPW; ++nt) {
+        float mx0 = fmaxf(x[nt][0], x[nt][2]), mx1 = fmaxf(x[nt][1], x[nt][3]);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = (mx0 > m0[nt] + kRescaleLog2) ? mx0 : m0[nt];
+        const float mn1 = (mx1 > m1[nt] + kRescaleLog2) ? mx1 : m1[nt];
+        const float al0 = fast_exp2(m0[nt] - mn0), al1 = fast_exp2(m1[nt] - mn1);  // -inf -> 0
+        l0[nt] *= al0;
+        l1[nt] *= al1;
+#pragma unroll
+        for (int mt = 0; mt < kMT; ++mt) {
+          o[nt][mt][0] *= al0;
+          o[nt][mt][1] *= al1;
+          o[nt][mt][2] *= al0;
+          o[nt][mt][3] *= al1;
+        }
+        m0[nt] = mn0;
+        m1[nt] = mn1;
       }
-      m0 = mn0;
-      m1 = mn1;
     }
-    uint32_t p01, p23;
-    if constexpr (!KV8) {
-      p01 = pack_bf16x2(fast_exp2(x0 - m0), fast_exp2(x1 - m1));
-      p23 = pack_bf16x2(fast_exp2(x2 - m0), fast_exp2(x3 - m1));
-      // the denominators sum the same bf16-rounded weights that multiply V
-      l0 += bf16lo_to_f32(p01) + bf16lo_to_f32(p23);
-      l1 += bf16hi_to_f32(p01) + bf16hi_to_f32(p23);
-    } else {
-      // f16 weights (<= 2^kRescaleLog2, in range) for the f16 P V product
-      p01 = pack_f16x2(fast_exp2(x0 - m0), fast_exp2(x1 - m1));
-      p23 = pack_f16x2(fast_exp2(x2 - m0), fast_exp2(x3 - m1));
-      l0 += f16lo_to_f32(p01) + f16lo_to_f32(p23);
-      l1 += f16hi_to_f32(p01) + f16hi_to_f32(p23);
+    uint32_t b0[TPW], b1[TPW];
+#pragma unroll
+    for (int nt = 0; nt < TPW; ++nt) {
+      uint32_t p01, p23;
+      if constexpr (!KV8) {
+        p01 = pack_bf16x2(fast_exp2(x[nt][0] - m0[nt]), fast_exp2(x[nt][1] - m1[nt]));
+        p23 = pack_bf16x2(fast_exp2(x[nt][2] - m0[nt]), fast_exp2(x[nt][3] - m1[nt]));
+        // the denominators sum the same bf16-rounded weights that multiply V
+        l0[nt] += bf16lo_to_f32(p01) + bf16lo_to_f32(p23);
+        l1[nt] += bf16hi_to_f32(p01) + bf16hi_to_f32(p23);
+      } else {
+        // f16 weights (<= 2^kRescaleLog2, in range) for the f16 P V product
+        p01 = pack_f16x2(fast_exp2(x[nt][0] - m0[nt]), fast_exp2(x[nt][1] - m1[nt]));
+        p23 = pack_f16x2(fast_exp2(x[nt][2] - m0[nt]), fast_exp2(x[nt][3] - m1[nt]));
+        l0[nt] += f16lo_to_f32(p01) + f16lo_to_f32(p23);
+        l1[nt] += f16hi_to_f32(p01) + f16hi_to_f32(p23);
+      }
+      // P^T as the B operand of the P V product
+      b0[nt] = movmatrix_trans(p01);
+      b1[nt] = movmatrix_trans(p23);
     }
 
-    // O^T (this warp's D rows x 8) += V^T (D rows x 16) * P^T (16 x 8)
-    const uint32_t b0 = movmatrix_trans(p01);
-    const uint32_t b1 = movmatrix_trans(p23);
+    // O^T (this warp's D rows x 8) += V^T (D rows x 16) * P^T (16 x 8) per head tile;
+    // each V fragment feeds every tile of the warp
     uint32_t vt[4];
     if constexpr (!KV8) {
 #pragma unroll
@@ -481,7 +547,8 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
       for (int mt = 0; mt < kMT; ++mt) {
         uint32_t a[4];
         ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
-        mma_bf16_16816(o[mt], a, b0, b1);
+#pragma unroll
+        for (int nt = 0; nt < TPW; ++nt) mma_bf16_16816(o[nt][mt], a, b0[nt], b1[nt]);
       }
     } else {
       // m-tile = one 16-byte chunk of D.  Transposed 8-bit loads give lane l the codes
@@ -496,10 +563,12 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
         ldmatrix_x4_trans(r, vt[mq & 3] + 128 * (mq >> 2));
         e4m3x4_to_f16x2x2(byte_perm(r[0], 0u, 0x3120u), a[0], a[1]);
         e4m3x4_to_f16x2x2(byte_perm(r[1], 0u, 0x3120u), a[2], a[3]);
-        mma_f16_16816(o[2 * mq], a, b0, b1);
+#pragma unroll
+        for (int nt = 0; nt < TPW; ++nt) mma_f16_16816(o[nt][2 * mq], a, b0[nt], b1[nt]);
         e4m3x4_to_f16x2x2(byte_perm(r[2], 0u, 0x3120u), a[0], a[1]);
         e4m3x4_to_f16x2x2(byte_perm(r[3], 0u, 0x3120u), a[2], a[3]);
-        mma_f16_16816(o[2 * mq + 1], a, b0, b1);
+#pragma unroll
+        for (int nt = 0; nt < TPW; ++nt) mma_f16_16816(o[nt][2 * mq + 1], a, b0[nt], b1[nt]);
       }
     }
   }
@@ -508,32 +577,39 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
 
   // ---- 4. merge the warps of each n8 tile and write ------------------------------------
 #pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  for (int nt = 0; nt < TPW; ++nt) {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0[nt] += __shfl_xor_sync(0xffffffffu, l0[nt], off);
+      l1[nt] += __shfl_xor_sync(0xffffffffu, l1[nt], off);
+    }
   }
   float* mbuf = reinterpret_cast<float*>(ring);
-  constexpr int kWarpFloats = 8 * kMergeStride + 16;
+  constexpr int kTileFloats = C::kTileFloats;   // [8 heads][kMergeStride] O, then m[8], l[8]
+  constexpr int kWarpFloats = TPW * kTileFloats;
   {
-    float* mine = mbuf + warp * kWarpFloats;
     const int g0 = 2 * (lane & 3);
     const int r8 = lane >> 2;
 #pragma unroll
-    for (int mt = 0; mt < kMT; ++mt) {
-      // rows r8 / r8 + 8 of the m-tile are d = 16 mt' + r8 / + 8 (bf16), or
-      // d = 16 mt' + 2 r8 / + 1 (E4M3 order)
-      constexpr int kHi = KV8 ? 1 : 8;
-      const int d = 16 * (wd * kMT + mt) + (KV8 ? 2 * r8 : r8);
-      mine[g0 * kMergeStride + d] = o[mt][0];
-      mine[(g0 + 1) * kMergeStride + d] = o[mt][1];
-      mine[g0 * kMergeStride + d + kHi] = o[mt][2];
-      mine[(g0 + 1) * kMergeStride + d + kHi] = o[mt][3];
-    }
-    if (r8 == 0) {
-      mine[8 * kMergeStride + g0] = m0;
-      mine[8 * kMergeStride + g0 + 1] = m1;
-      mine[8 * kMergeStride + 8 + g0] = l0;
-      mine[8 * kMergeStride + 8 + g0 + 1] = l1;
+    for (int nt = 0; nt < TPW; ++nt) {
+      float* mine = mbuf + warp * kWarpFloats + nt * kTileFloats;
+#pragma unroll
+      for (int mt = 0; mt < kMT; ++mt) {
+        // rows r8 / r8 + 8 of the m-tile are d = 16 mt' + r8 / + 8 (bf16), or
+        // d = 16 mt' + 2 r8 / + 1 (E4M3 order)
+        constexpr int kHi = KV8 ? 1 : 8;
+        const int d = 16 * (wd * kMT + mt) + (KV8 ? 2 * r8 : r8);
+        mine[g0 * kMergeStride + d] = o[nt][mt][0];
+        mine[(g0 + 1) * kMergeStride + d] = o[nt][mt][1];
+        mine[g0 * kMergeStride + d + kHi] = o[nt][mt][2];
+        mine[(g0 + 1) * kMergeStride + d + kHi] = o[nt][mt][3];
+      }
+      if (r8 == 0) {
+        mine[8 * kMergeStride + g0] = m0[nt];
+        mine[8 * kMergeStride + g0 + 1] = m1[nt];
+        mine[8 * kMergeStride + 8 + g0] = l0[nt];
+        mine[8 * kMergeStride + 8 + g0 + 1] = l1[nt];
+      }
     }
   }
   __syncthreads();
@@ -543,19 +619,21 @@ __global__ void __launch_bounds__(32 * NTILE * DSPLIT * SL, MINB)
     const int dg = it & 31;  // 8-wide d group
     if (gg >= G) continue;
     const int nt = gg >> 3, g = gg & 7;
-    // the warps holding this (head, d) range: one per slot lane
-    const int part = NTILE > 1 ? nt : (dg * 8) / (kHeadDim / DSPLIT);
+    // the warps holding this (head, d) range, one per slot lane: the D-half's warp
+    // (tile record nt) or the tile's warp (its only record)
+    const int part = DSPLIT > 1 ? (dg * 8) / (kHeadDim / DSPLIT) : nt;
+    const int trec = DSPLIT > 1 ? nt * kTileFloats : 0;
     float mstar = kNegInf;
 #pragma unroll
     for (int w = 0; w < SL; ++w)
-      mstar = fmaxf(mstar, mbuf[(part * SL + w) * kWarpFloats + 8 * kMergeStride + g]);
+      mstar = fmaxf(mstar, mbuf[(part * SL + w) * kWarpFloats + trec + 8 * kMergeStride + g]);
     float lsum = 0.f;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
     for (int w = 0; w < SL; ++w) {
-      const float* src = mbuf + (part * SL + w) * kWarpFloats;
+      const float* src = mbuf + (part * SL + w) * kWarpFloats + trec;
       const float sc = fast_exp2(src[8 * kMergeStride + g] - mstar);  // -inf -> 0
       lsum += sc * src[8 * kMergeStride + 8 + g];
       const float4 a = *reinterpret_cast<const float4*>(src + g * kMergeStride + dg * 8);
@@ -683,12 +761,16 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
 #define QSA_FP8_LARGE_SL 3
 #endif
 #ifndef QSA_FP8_LARGE_STAGES
-#define QSA_FP8_LARGE_STAGES 3
+#define QSA_FP8_LARGE_STAGES 4
 #endif
 using CfgSmall = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES>;
-using CfgLarge = Cfg<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES>;
+#ifndef QSA_LARGE_DSPLIT
+#define QSA_LARGE_DSPLIT 2  // 8 < G <= 16: the pair splits D (2) or the head tiles (1)
+#endif
+constexpr bool kLargeQsplit = QSA_LARGE_DSPLIT == 2;
+using CfgLarge = Cfg<2, QSA_LARGE_DSPLIT, QSA_LARGE_SL, QSA_LARGE_STAGES>;
 using CfgSmall8 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true>;
-using CfgLarge8 = Cfg<2, 1, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, true>;
+using CfgLarge8 = Cfg<2, QSA_LARGE_DSPLIT, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, true>;
 static_assert(CfgSmall::kSmem <= CfgSmall::kSmPerCta(QSA_SMALL_CTAS), "small shape: CTAs per SM");
 static_assert(CfgLarge::kSmem <= CfgLarge::kSmPerCta(QSA_LARGE_CTAS), "large shape: CTAs per SM");
 static_assert(CfgSmall8::kSmem <= CfgSmall8::kSmPerCta(QSA_SMALL_CTAS), "E4M3 small shape: CTAs per SM");
@@ -720,13 +802,13 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   if (p.kv_fp8) {
     e = (p.G <= 8) ? launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
                                 true>(p, stream)
-                   : launch_fwd<2, 1, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, QSA_LARGE_CTAS, false,
-                                true>(p, stream);
+                   : launch_fwd<2, QSA_LARGE_DSPLIT, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES,
+                                QSA_LARGE_CTAS, kLargeQsplit, true>(p, stream);
   } else {
     e = (p.G <= 8) ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
                                 QSA_SMALL_QSPLIT, false>(p, stream)
-                   : launch_fwd<2, 1, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS, false, false>(
-                         p, stream);
+                   : launch_fwd<2, QSA_LARGE_DSPLIT, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS,
+                                kLargeQsplit, false>(p, stream);
   }
   if (e != cudaSuccess || p.nsplit == 1) return e;
   const int64_t rows = int64_t(p.Tq) * p.Hq;

@@ -7,7 +7,9 @@
 // over the selected slots only and return P V; a row without a valid slot returns 0.
 //
 // K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit, two CTAs
-// resident per SM so that one CTA's prologue and epilogue overlap the other's gather:
+// resident per SM so that one CTA's prologue and epilogue overlap the other's gather
+// (units ordered KV head slowest when one head's slice of the cache fits L2 and the
+// whole cache does not):
 //   1. stage the split's slot indices in shared memory and compact away -1 (and
 //      out-of-range) entries with a block scan, so masked slots cost no bandwidth;
 //   2. gather K and V rows of the compacted slots with 16-byte cp.async into shared
@@ -19,8 +21,8 @@
 //   3. per slot lane and 16-slot sub-tile: S^T = K Q^T with the slots as the MMA M
 //      dimension and the (up to 8) heads of one n8 tile as N, so the group shares every
 //      gathered row and G = 3/6/8/12/16 needs no padding of the head ratio in memory
-//      (G <= 8: the pair splits D for both products and exchanges partial scores;
-//      G > 8: the pair splits the two head tiles); online softmax in fp32 registers
+//      (the warp pair splits D for both products and exchanges partial scores; for
+//      G > 8 each warp handles both n8 head tiles); online softmax in fp32 registers
 //      (base 2, lazy rescaling); P rounded to bf16 and transposed in registers
 //      (movmatrix) into the B operand of O^T += V^T P^T with D = 256 as M;
 //   4. merge the per-warp (m, l, O) states through shared memory and write bf16 out

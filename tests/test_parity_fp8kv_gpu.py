@@ -237,3 +237,12 @@ def test_from_host_and_graph_capture(cuda_device, oracle_lib):
     torch.cuda.synchronize()
     compare(w, o.cpu(), oracle_lib, 1.0 / 16.0, None, "e4m3 graph replay")
     del graph
+
+
+def test_long_prefill_all_rows_in_convex_hull(cuda_device):
+    """Every output element of the full-size E4M3 long prefill lies between the minimum and
+    the maximum of its selected dequantised V elements (up to the output's bf16 rounding)."""
+    from test_parity_gpu import _convex_hull_all_rows
+    w = wl.long_prefill_e4m3kv()
+    got = run(w, dev(w, cuda_device), 1.0 / 16.0)
+    _convex_hull_all_rows(w, got, v_scale=w.v_scale)

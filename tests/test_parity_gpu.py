@@ -498,3 +498,31 @@ def test_very_wide_selection(cuda_device, oracle_lib):
     got = run(dev(w, cuda_device), 1.0 / 16.0)
     rows = list(range(0, 40, 3))
     compare_rows(w, got, oracle_lib, 1.0 / 16.0, rows, "W=20000")
+
+
+def _convex_hull_all_rows(w, got, v_scale=1.0, chunk=128):
+    """Every output element is a convex combination of the selected V rows' elements:
+    it lies between their minimum and maximum for that (KV head, d), up to the bf16
+    rounding of the output.  Checked for every row and head at full size on the GPU
+    (torch gathers; the product path is not involved)."""
+    dev = torch.device("cuda", 0)
+    v = w.v_cache.to(dev)
+    vf = (v.float() * v_scale) if v.dtype == torch.float8_e4m3fn else v.float()
+    G = w.Hq // w.Hkv
+    out = got.to(dev).float().view(w.Tq, w.Hkv, G, D)
+    for r0 in range(0, w.Tq, chunk):
+        idx = w.slot_idx[r0:r0 + chunk].to(dev).long()
+        valid = idx >= 0
+        rows = vf[idx.clamp_min(0)]                            # [c, W, Hkv, D]
+        big = torch.finfo(torch.float32).max
+        lo = torch.where(valid[..., None, None], rows, big).amin(dim=1)    # [c, Hkv, D]
+        hi = torch.where(valid[..., None, None], rows, -big).amax(dim=1)
+        o = out[r0:r0 + chunk]                                   # [c, Hkv, G, D]
+        tol = 2.0 ** -7 * torch.maximum(lo.abs(), hi.abs())[:, :, None, :] + 1e-6
+        assert (o >= lo[:, :, None, :] - tol).all() and (o <= hi[:, :, None, :] + tol).all(), r0
+
+
+def test_long_prefill_all_rows_in_convex_hull(cuda_device):
+    w = wl.long_prefill()
+    got = run(dev(w, cuda_device), 1.0 / 16.0)
+    _convex_hull_all_rows(w, got)

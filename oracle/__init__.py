@@ -8,8 +8,10 @@ The arithmetic lives in ``qsa_oracle.c`` (plain C, fp32, OpenMP over query rows)
 follows the article "Qwen4-Exp QSA comes to Huawei's Ascend: inside SGLang's opt-in
 CANN prefill PR", section "What the pull request actually adds" (softmax(scale*QK^T)V
 over the selected slots, -1 masked, fully masked rows zero) and section "Nine tests
-that passed, ..." (FP32 CPU reference from the same BF16 inputs).  This module only
-compiles that file with gcc and marshals numpy / torch CPU arrays into it.
+that passed, ..." (FP32 CPU reference from the same BF16 inputs), plus block selection
+and the fp8_e4m3 KV cache (sections "Why QSA is the awkward part, in numbers" and "Where
+this sits in the Qwen4Exp serving build-out").  This module only compiles that file with
+gcc and marshals numpy / torch CPU arrays into it.
 """
 from __future__ import annotations
 

@@ -15,6 +15,10 @@
  *     rows output zero ("zero-output convention").
  *   - "Nine tests that passed, ...": an FP32 CPU reference computed from the same BF16
  *     inputs; unordered physical slots; zero selection width.
+ *   - "Why QSA is the awkward part, in numbers": block selection ("block4"), see
+ *     qsa_oracle_forward_block.
+ *   - "Where this sits in the Qwen4Exp serving build-out": the fp8_e4m3 KV cache, see
+ *     qsa_oracle_forward_fp8kv (E4M3 decoded field by field from the format's definition).
  * Precision: the article fixes FP32 for the reference, so every accumulation below is
  * a float in plain sequential order.  exp is the C library's expf.
  *

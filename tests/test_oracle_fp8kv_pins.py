@@ -8,6 +8,8 @@ per tensor, dequantised value = code value x scale, then the plain attention def
 Pins:
   * the E4M3 decoder against hand-worked code values (tests/golden/e4m3_codes.json) and
     against torch's float8_e4m3fn conversion for all 256 codes (a library routine);
+  * hand-worked forward cases (tests/golden/e4m3_forward_cases.json: weights 3/4 and 1/4
+    from a ln 3 score gap, subnormal and negative codes with scales);
   * with power-of-two scales every dequantised element is exactly a bf16 value, so the
     fp8 path must reproduce the (separately pinned) bf16 oracle on those bf16 tensors;
   * float64 brute force on tiny inputs with general scales (decoded by torch);
@@ -181,8 +183,47 @@ def pin_error_flags(o):
     assert err & 2
 
 
-PINS = [pin_decode_golden, pin_decode_library, pin_matches_bf16_oracle, pin_brute_force,
-        pin_closed_forms, pin_block_selection, pin_error_flags]
+FORWARD_GOLDEN = Path(__file__).resolve().parent / "golden" / "e4m3_forward_cases.json"
+_SCALES = {"ln3": math.log(3.0), "ln2": math.log(2.0), "1": 1.0}
+
+
+def load_forward_golden():
+    """The hand-worked fp8 forward cases: bf16 q, E4M3 code caches, expected outputs."""
+    spec = json.loads(FORWARD_GOLDEN.read_text())
+    cases = []
+    for c in spec["cases"]:
+        Tq, Hq, Hkv, S = c["Tq"], c["Hq"], c["Hkv"], c["S"]
+        q = torch.zeros(Tq, Hq, D)
+        for t, h, d, val in c["q"]:
+            q[t, h, d] = val
+        kc = torch.zeros(S, Hkv, D, dtype=torch.uint8)
+        for s_, j, d, code in c["k_codes"]:
+            kc[s_, j, d] = int(code, 16)
+        vc = torch.zeros(S, Hkv, D, dtype=torch.uint8)
+        for s_, j, d, code in c["v_codes"]:
+            vc[s_, j, d] = int(code, 16)
+        exp = torch.zeros(Tq, Hq, D, dtype=torch.float64)
+        for t, h, d, val in c["expected"]:
+            exp[t, h, d] = val
+        cases.append(dict(name=c["name"], q=q.to(torch.bfloat16), k=kc, v=vc,
+                          slot_idx=torch.tensor(c["slot_idx"], dtype=torch.int32),
+                          scale=_SCALES[c["scale"]], k_scale=c["k_scale"], v_scale=c["v_scale"],
+                          expected=exp))
+    return cases
+
+
+def pin_forward_golden(o):
+    for c in load_forward_golden():
+        got = o.forward_fp8kv(c["q"], c["k"], c["v"], c["slot_idx"], None, c["scale"],
+                              c["k_scale"], c["v_scale"])
+        np.testing.assert_allclose(got, c["expected"].numpy(), rtol=0, atol=2e-6, err_msg=c["name"])
+        empty = (c["expected"].abs().sum(dim=(1, 2)) == 0).nonzero().flatten().tolist()
+        for t in empty:
+            assert np.all(got[t] == 0) and not np.signbit(got[t]).any(), c["name"]
+
+
+PINS = [pin_decode_golden, pin_decode_library, pin_forward_golden, pin_matches_bf16_oracle,
+        pin_brute_force, pin_closed_forms, pin_block_selection, pin_error_flags]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)

@@ -246,3 +246,18 @@ def test_long_prefill_all_rows_in_convex_hull(cuda_device):
     w = wl.long_prefill_e4m3kv()
     got = run(w, dev(w, cuda_device), 1.0 / 16.0)
     _convex_hull_all_rows(w, got, v_scale=w.v_scale)
+
+
+def test_forward_golden(cuda_device):
+    """The hand-worked fp8 forward cases (tests/golden/e4m3_forward_cases.json) through the
+    CUDA path, against their exact expected values."""
+    from test_oracle_fp8kv_pins import load_forward_golden
+    for c in load_forward_golden():
+        out = qsa.sparse_prefill(c["q"].to(cuda_device),
+                                 c["k"].view(torch.float8_e4m3fn).to(cuda_device),
+                                 c["v"].view(torch.float8_e4m3fn).to(cuda_device),
+                                 c["slot_idx"].to(cuda_device), scale=c["scale"],
+                                 k_scale=c["k_scale"], v_scale=c["v_scale"])
+        torch.cuda.synchronize()
+        empty = (c["expected"].abs().sum(dim=(1, 2)) == 0).nonzero().flatten().tolist()
+        check_gates(out.float().cpu(), c["expected"], empty, "e4m3 golden: " + c["name"])

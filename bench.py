@@ -200,8 +200,19 @@ def cpu_baseline(w: wl.Workload, target_s: float):
     dt = time.perf_counter() - t0
     flops = int(pairs_per_row(w)[:n].sum()) * w.Hq * 4 * 256
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": o.num_threads(),
+            "nproc": os.cpu_count(), "cpu_model": _cpu_model(),
             "kind": "oracle", "seconds": round(dt, 3),
             "sample": f"first {n} of {w.Tq} query rows of the same workload (all heads, all selected slots)"}
+
+
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, rank):
@@ -235,6 +246,7 @@ def run_reference(args, rank):
         "config": {"workload": w.name, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": 256, "S": w.S,
                    "W": w.W, "valid_pairs": pairs, "parallelism": "replicas"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": o.num_threads(),
+                         "nproc": os.cpu_count(), "cpu_model": _cpu_model(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))

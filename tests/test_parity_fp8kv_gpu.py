@@ -95,7 +95,8 @@ def test_width_sweep(cuda_device, oracle_lib, scale, nsplit):
     compare(w, got, oracle_lib, scale, None, f"e4m3 width_sweep s={scale}")
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (24, 2), (12, 1), (6, 1), (3, 1), (16, 1), (5, 1), (2, 2)])
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (24, 2), (12, 1), (6, 1), (3, 1), (16, 1), (5, 1), (2, 2),
+                                    (10, 1), (32, 2)])
 @pytest.mark.parametrize("Tq", [1, 257])
 def test_head_shapes(cuda_device, oracle_lib, Hq, Hkv, Tq):
     """Both kernel shapes (G <= 8 and G > 8), ragged widths and interior -1s."""
@@ -261,3 +262,19 @@ def test_forward_golden(cuda_device):
         torch.cuda.synchronize()
         empty = (c["expected"].abs().sum(dim=(1, 2)) == 0).nonzero().flatten().tolist()
         check_gates(out.float().cpu(), c["expected"], empty, "e4m3 golden: " + c["name"])
+
+
+def test_strided_kv_and_out_views(cuda_device, oracle_lib):
+    """E4M3 K and V as views into one [S, 2, Hkv, D] code buffer (byte strides); out as a
+    view of a wider buffer."""
+    w = _random_case(2700, 100, 16, 2, 2048, 300, minus1=0.1)
+    kv = torch.stack([w.k_cache.view(torch.uint8), w.v_cache.view(torch.uint8)], dim=1)
+    kv = kv.view(torch.float8_e4m3fn).to(cuda_device)                  # [S, 2, Hkv, D]
+    big = torch.zeros(100, 16, 2 * D, dtype=torch.bfloat16, device=cuda_device)
+    out = big[:, :, D:]
+    assert not out.is_contiguous() and not kv[:, 0].is_contiguous()
+    qsa.sparse_prefill(w.q.to(cuda_device), kv[:, 0], kv[:, 1], w.slot_idx.to(cuda_device),
+                       scale=1.0 / 16.0, out=out, k_scale=w.k_scale, v_scale=w.v_scale)
+    torch.cuda.synchronize()
+    compare(w, out.cpu(), oracle_lib, 1.0 / 16.0, None, "e4m3 strided views")
+    assert (big[:, :, :D] == 0).all()

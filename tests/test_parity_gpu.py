@@ -154,7 +154,8 @@ def _random_case(seed, Tq, Hq, Hkv, S, W, minus1=0.0, widths=False):
     return wl.Workload(f"rand_{Hq}_{Hkv}_{Tq}", q, k, v, idx, width)
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (24, 2), (12, 1), (6, 1), (3, 1), (16, 1), (5, 1), (2, 2)])
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (24, 2), (12, 1), (6, 1), (3, 1), (16, 1), (5, 1), (2, 2),
+                                    (10, 1), (32, 2)])
 @pytest.mark.parametrize("Tq", [1, 257])
 def test_head_shapes(cuda_device, oracle_lib, Hq, Hkv, Tq):
     w = _random_case(1000 + Hq * 10 + Hkv + Tq, Tq, Hq, Hkv, 8192, 2051, minus1=0.05, widths=True)

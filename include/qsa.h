@@ -204,6 +204,60 @@ qsa_status_t qsa_sparse_prefill_fp8kv(const void* q, int64_t q_stride_t, int64_t
                                       void* workspace, size_t workspace_bytes,
                                       uint32_t* err_word, void* stream);
 
+/*
+ * qsa_sparse_prefill_partial / qsa_combine_partials -- context parallelism: the K/V cache
+ * split by slot range across devices.
+ *
+ * Source: the article "Qwen4-Exp QSA comes to Huawei's Ascend: inside SGLang's opt-in
+ * CANN prefill PR", section "Where this sits in the Qwen4Exp serving build-out", which
+ * names decode context parallelism (DCP) for this attention path.  Reading taken here:
+ * device r holds the global slots [slot_lo_r, slot_lo_r + S_r) of the cache; every device
+ * sees the same (global) selection; each computes, over its own slots only, the
+ * softmax-normalised output and the log-sum-exp of its scores; the records of all devices
+ * are exchanged (an all-gather) and combined with log-sum-exp weights, which gives exactly
+ * the attention over the union of the slots (the same combine as the split-W path).
+ *
+ * qsa_sparse_prefill_partial: arguments as qsa_sparse_prefill_block (kv_fp8 = 0, bf16
+ * caches) or qsa_sparse_prefill_fp8kv (kv_fp8 = 1, E4M3 caches with k_scale / v_scale),
+ * except:
+ *   k_cache, v_cache   this device's slots only: row s of the tensors is global slot
+ *                      slot_lo + s, 0 <= s < S.
+ *   slot_lo            first global slot held here, a non-negative multiple of block
+ *                      (any value <= S_total for an empty shard, S == 0).
+ *   S_total            global slot extent (>= slot_lo + S).  Selected entries in
+ *                      [0, S_total) outside this device's range are skipped silently;
+ *                      entries outside [-1, S_total) set QSA_ERRBIT_SLOT_RANGE.
+ *   part_o             fp32 [Tq, Hq, D] contiguous (16-byte aligned): the output
+ *                      normalised over this device's valid slots (zeros where it has none).
+ *   part_lse           fp32 [Tq, Hq] contiguous: log2 of the sum over this device's valid
+ *                      slots of 2^(scale * log2(e) * s_i) (k_scale included for E4M3), i.e.
+ *                      the base-2 log-sum-exp of the scaled scores; -inf where none.
+ * The split plan and workspace are those of qsa_sparse_prefill_block_plan; the device's
+ * own splits are combined into the one record before the call's work ends.
+ *
+ * qsa_combine_partials: out[t, h, :] = sum_r 2^(lse_r - m) O_r / sum_r 2^(lse_r - m),
+ * m = max_r lse_r, over R records stacked as part_o [R, Tq, Hq, D] and part_lse
+ * [R, Tq, Hq] (the layout an all-gather of the records produces); records with
+ * lse = -inf weigh 0; a row with no record above -inf is written as exact zeros.  out is
+ * bf16 [Tq, Hq, D] with strides (out_stride_t, out_stride_h, 1), multiples of 8.
+ * Both entry points enqueue on `stream` only and allocate nothing.
+ */
+qsa_status_t qsa_sparse_prefill_partial(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                        const void* k_cache, int64_t k_stride_s,
+                                        int64_t k_stride_h, const void* v_cache,
+                                        int64_t v_stride_s, int64_t v_stride_h,
+                                        const int32_t* slot_idx, int64_t idx_stride_t,
+                                        const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                        int32_t D, int64_t S, int32_t W, int32_t block,
+                                        int64_t slot_lo, int64_t S_total, int32_t kv_fp8,
+                                        float scale, float k_scale, float v_scale, float* part_o,
+                                        float* part_lse, int32_t nsplit, void* workspace,
+                                        size_t workspace_bytes, uint32_t* err_word, void* stream);
+
+qsa_status_t qsa_combine_partials(const float* part_o, const float* part_lse, int32_t R,
+                                  int32_t Tq, int32_t Hq, int32_t D, void* out,
+                                  int64_t out_stride_t, int64_t out_stride_h, void* stream);
+
 /* Size of the device scratch array that qsa_sparse_prefill_noalloc uses (16 MiB). */
 #define QSA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 

@@ -229,3 +229,68 @@ def test_wrapper_refuses_cpu_fp8_tensors():
     idx = torch.zeros(2, 3, dtype=torch.int32)
     with pytest.raises(ValueError):
         qsa.sparse_prefill(q, k, k, idx, k_scale=0.5, v_scale=0.5)
+
+
+def _call_partial(**over):
+    """A raw call of the slot-range partial entry point with fake aligned pointers."""
+    a = dict(q=0x10000, q_stride_t=16 * 256, q_stride_h=256, k_cache=0x20000, k_stride_s=512,
+             k_stride_h=256, v_cache=0x30000, v_stride_s=512, v_stride_h=256, slot_idx=0x40000,
+             idx_stride_t=8, width=None, Tq=4, Hq=16, Hkv=2, D=256, S=100, W=8, block=1,
+             slot_lo=0, S_total=100, kv_fp8=0, scale=0.0625, k_scale=1.0, v_scale=1.0,
+             part_o=0x50000, part_lse=0x60000, nsplit=1, workspace=None, workspace_bytes=0,
+             err_word=None, stream=None)
+    a.update(over)
+    return qsa.qsa_sparse_prefill_partial(**a)
+
+
+INVALID_PARTIAL = [
+    (dict(part_o=None), qsa.QSA_ERR_INVALID_ARG),
+    (dict(part_lse=None), qsa.QSA_ERR_INVALID_ARG),
+    (dict(part_o=0x50004), qsa.QSA_ERR_INVALID_ARG),          # misaligned record
+    (dict(slot_lo=-8), qsa.QSA_ERR_INVALID_ARG),
+    (dict(slot_lo=6, block=4, S=96, S_total=200), qsa.QSA_ERR_INVALID_ARG),   # not a block multiple
+    (dict(slot_lo=50, S_total=120), qsa.QSA_ERR_INVALID_ARG),  # S_total < slot_lo + S
+    (dict(S_total=-1), qsa.QSA_ERR_INVALID_ARG),
+    (dict(kv_fp8=2), qsa.QSA_ERR_INVALID_ARG),
+    (dict(D=128), qsa.QSA_ERR_UNSUPPORTED),
+    (dict(k_cache=None), qsa.QSA_ERR_INVALID_ARG),            # S > 0 needs the caches
+]
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="fake-pointer validation runs only where no GPU can be reached")
+@pytest.mark.parametrize("over,status", INVALID_PARTIAL, ids=[str(o) for o, _ in INVALID_PARTIAL])
+def test_partial_invalid_arguments_rejected_before_launch(lib, over, status):
+    assert _call_partial(**over) == status
+    assert qsa.qsa_last_error_detail() != ""
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_partial_valid_shard_reaches_the_device_query(lib):
+    # a shard in the middle of the cache, E4M3 caches, and an empty shard with NULL caches
+    assert _call_partial(slot_lo=100, S=50, S_total=400, nsplit=0) == qsa.QSA_ERR_CUDA
+    assert _call_partial(kv_fp8=1, k_scale=0.5, v_scale=0.25, nsplit=0) == qsa.QSA_ERR_CUDA
+    assert _call_partial(S=0, slot_lo=100, k_cache=None, v_cache=None, nsplit=0) == qsa.QSA_ERR_CUDA
+    assert _call_partial(Tq=0, q=None, part_o=None, part_lse=None) == qsa.QSA_OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="fake-pointer validation runs only where no GPU can be reached")
+def test_combine_partials_validation(lib):
+    ok = dict(part_o=0x50000, part_lse=0x60000, R=2, Tq=4, Hq=16, D=256, out=0x70000,
+              out_stride_t=16 * 256, out_stride_h=256, stream=None)
+    bad = [dict(R=0), dict(Hq=0), dict(Tq=-1), dict(part_o=None), dict(out=None),
+           dict(part_o=0x50008), dict(out_stride_h=12)]
+    for over in bad:
+        assert qsa.qsa_combine_partials(**{**ok, **over}) == qsa.QSA_ERR_INVALID_ARG, over
+    assert qsa.qsa_combine_partials(**{**ok, "D": 128}) == qsa.QSA_ERR_UNSUPPORTED
+    assert qsa.qsa_combine_partials(**{**ok, "Tq": 0, "part_o": None}) == qsa.QSA_OK
+    assert qsa.qsa_combine_partials(**ok) == qsa.QSA_ERR_CUDA   # valid: the launch fails
+
+
+def test_shard_ranges():
+    assert qsa.shard_ranges(65536, 2) == [(0, 32768), (32768, 65536)]
+    r = qsa.shard_ranges(1000, 3, block=4)
+    assert r[0][0] == 0 and r[-1][1] == 1000
+    assert all(lo % 4 == 0 for lo, _ in r) and all(a[1] == b[0] for a, b in zip(r, r[1:]))
+    assert qsa.shard_ranges(10, 4, block=4)[-1] == (10, 10)   # more ranks than blocks

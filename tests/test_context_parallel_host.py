@@ -1,0 +1,127 @@
+"""Host side of context parallelism (the cache split by slot range across ranks): the
+shard ranges and the exchange of the ranks' partial records, run as world-size-2 and 3
+gloo process groups on the CPU.  The kernels are replaced by exact float64 restatements
+of what the entry points document (the record: output normalised over the rank's valid
+slots and the base-2 log-sum-exp of their scaled scores; the combine: log-sum-exp
+weights), so the test checks the sharding and the exchange order; the result must equal
+the CPU oracle on the whole cache.  The CUDA records and combine are checked on the GPU
+in test_parity_gpu.py."""
+from __future__ import annotations
+
+import datetime
+import math
+import os
+import socket
+import sys
+from pathlib import Path
+
+import numpy as np
+import torch
+import torch.multiprocessing as mp
+
+ROOT = Path(__file__).resolve().parent.parent
+sys.path.insert(0, str(ROOT))
+
+from top_sparse_attention_index_b200 import context_parallel as cp  # noqa: E402
+from top_sparse_attention_index_b200 import workloads as wl  # noqa: E402
+
+D = 256
+
+
+def _case():
+    g = torch.Generator().manual_seed(91)
+    Tq, Hq, Hkv, S, W = 6, 8, 2, 120, 40
+    q = torch.randn(Tq, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    idx = wl.uniform_distinct(g, Tq, S, W)
+    idx[1, :] = -1                         # a fully masked row
+    idx[2, 5:] = idx[2, 5:].clamp(max=20)  # row 2 mostly in the first shard
+    return q, k, v, idx
+
+
+def _partial_double(q, k_local, v_local, slot_idx, slot_lo, S_total, width=None, scale=None,
+                    block=1, k_scale=1.0, v_scale=1.0):
+    """float64 restatement of qsa_sparse_prefill_partial's documented record."""
+    scale = 1.0 / 16.0 if scale is None else scale
+    Tq, Hq, _ = q.shape
+    S_loc, Hkv, _ = k_local.shape
+    G = Hq // Hkv
+    o = np.zeros((Tq, Hq, D), dtype=np.float32)
+    lse = np.full((Tq, Hq), -np.inf, dtype=np.float32)
+    qd, kd, vd = q.double().numpy(), k_local.double().numpy(), v_local.double().numpy()
+    for t in range(Tq):
+        sel = [int(s) - slot_lo for s in slot_idx[t] if slot_lo <= int(s) < slot_lo + S_loc]
+        if not sel:
+            continue
+        for h in range(Hq):
+            x = scale * math.log2(math.e) * (kd[sel, h // G] @ qd[t, h])
+            m = x.max()
+            p = np.exp2(x - m)
+            o[t, h] = (p @ vd[sel, h // G]) / p.sum()
+            lse[t, h] = m + math.log2(p.sum())
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def _combine_double(g_o, g_l, out=None):
+    o, l = g_o.double().numpy(), g_l.double().numpy()
+    m = l.max(axis=0)
+    w = np.where(np.isfinite(l), np.exp2(l - np.where(np.isfinite(m), m, 0)), 0.0)
+    num = (w[..., None] * np.nan_to_num(o)).sum(axis=0)
+    den = w.sum(axis=0)
+    return torch.from_numpy(np.where(den[..., None] > 0, num / np.maximum(den, 1e-300)[..., None], 0.0))
+
+
+def _rank_main(rank, world, port, queue):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    q, k, v, idx = _case()
+    S = k.shape[0]
+    lo, hi = cp.shard_ranges(S, world)[rank]
+    out = cp.sparse_prefill_context_parallel(q, k[lo:hi], v[lo:hi], idx, lo, S,
+                                             partial_fn=_partial_double,
+                                             combine_fn=_combine_double)
+    queue.put((rank, out.numpy()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _run(world):
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, queue)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = dict(queue.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return results
+
+
+def test_context_parallel_exchange_matches_the_whole_cache(oracle_lib):
+    q, k, v, idx = _case()
+    ref = oracle_lib.forward(q, k, v, idx, None, 1.0 / 16.0)
+    for world in (2, 3):
+        results = _run(world)
+        for r in range(world):
+            np.testing.assert_allclose(results[r], ref, rtol=1e-5, atol=1e-6)
+        assert np.all(results[0][1] == 0)   # the fully masked row
+
+
+def test_shard_ranges_cover_the_cache_once():
+    for S, world, block in ((65536, 8, 1), (1000, 3, 4), (7, 2, 1), (10, 4, 4)):
+        r = cp.shard_ranges(S, world, block)
+        assert len(r) == world and r[0][0] == 0 and r[-1][1] == S
+        assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
+        assert all(hi >= lo and (lo % block == 0 or hi == lo) for lo, hi in r)

@@ -278,3 +278,11 @@ def test_strided_kv_and_out_views(cuda_device, oracle_lib):
     torch.cuda.synchronize()
     compare(w, out.cpu(), oracle_lib, 1.0 / 16.0, None, "e4m3 strided views")
     assert (big[:, :, :D] == 0).all()
+
+
+def test_context_parallel_shards(cuda_device, oracle_lib):
+    """E4M3 cache split by slot range over 3 emulated ranks: records stacked and combined."""
+    from test_parity_gpu import _shards_combined
+    w = _random_case(2800, 200, 16, 2, 16384, 2051, minus1=0.05, widths=True)
+    got, _ = _shards_combined(w, dev(w, cuda_device), 3, k_scale=w.k_scale, v_scale=w.v_scale)
+    compare(w, got, oracle_lib, 1.0 / 16.0, None, "e4m3 context parallel R=3")

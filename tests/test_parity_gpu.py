@@ -527,3 +527,66 @@ def test_long_prefill_all_rows_in_convex_hull(cuda_device):
     w = wl.long_prefill()
     got = run(dev(w, cuda_device), 1.0 / 16.0)
     _convex_hull_all_rows(w, got)
+
+
+# ---- context parallelism: slot-range shards emulated on one device ----------------------
+
+def _shards_combined(w, d, R, scale=1.0 / 16.0, nsplit=0, **kw):
+    """Every shard's partial record (one device standing in for R ranks, one after
+    another), stacked as an all-gather would and combined."""
+    rec_o, rec_l = [], []
+    for lo, hi in qsa.shard_ranges(w.S, R, w.block):
+        po, pl = qsa.sparse_prefill_partial(d["q"], d["k_cache"][lo:hi], d["v_cache"][lo:hi],
+                                            d["slot_idx"], lo, w.S, width=d["width"],
+                                            scale=scale, nsplit=nsplit, block=w.block, **kw)
+        rec_o.append(po)
+        rec_l.append(pl)
+    out = qsa.combine_partials(torch.stack(rec_o), torch.stack(rec_l))
+    torch.cuda.synchronize()
+    return out.cpu(), rec_l
+
+
+@pytest.mark.parametrize("R", [1, 2, 3, 5])
+def test_context_parallel_shards(cuda_device, oracle_lib, R):
+    w = _random_case(90 + R, 300, 16, 2, 16384, 2051, minus1=0.05, widths=True)
+    d = dev(w, cuda_device)
+    got, rec_l = _shards_combined(w, d, R)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"context parallel R={R}")
+    if R == 1:  # one shard holding the whole cache: bitwise the unsharded call
+        assert torch.equal(got.view(torch.int16), run(d, 1.0 / 16.0).view(torch.int16))
+    for t in empty_rows(w):
+        assert all(torch.isinf(l[t]).all() for l in rec_l)
+
+
+def test_context_parallel_wide_rows_and_decode(cuda_device, oracle_lib):
+    """W = 6,000 (each shard combines its own splits into one record) and a decode-shape
+    batch with forced split counts."""
+    w = _random_case(95, 120, 16, 2, 20000, 6000, minus1=0.1, widths=True)
+    got, _ = _shards_combined(w, dev(w, cuda_device), 3)
+    rows = list(range(0, w.Tq, 4))
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0, rows=rows)
+    check_gates(got[rows].float(), torch.from_numpy(ref), empty_rows(w, rows), "context parallel W=6000")
+    w = _random_case(96, 3, 16, 2, 65536, 2051, minus1=0.2)
+    for nsplit in (1, 4, 16):
+        got, _ = _shards_combined(w, dev(w, cuda_device), 2, nsplit=nsplit)
+        ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
+        check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"context parallel decode n={nsplit}")
+
+
+def test_context_parallel_block4_and_empty_shard(cuda_device, oracle_lib):
+    """Block selection with shard boundaries on block multiples, and more ranks than
+    blocks (the last shard is empty: NULL-free zero-row caches, a record of -inf)."""
+    w = _random_case(97, 64, 16, 2, 4096, 300, minus1=0.1)
+    w.slot_idx = wl.uniform_distinct(torch.Generator().manual_seed(98), 64, 1024, 300)
+    w.block = 4
+    got, _ = _shards_combined(w, dev(w, cuda_device), 3)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0, block=4)
+    check_gates(got.float(), torch.from_numpy(ref), None, "context parallel block4")
+    t = _random_case(99, 8, 16, 2, 12, 10, minus1=0.0)
+    t.block = 4  # 3 blocks over 4 ranks
+    t.slot_idx = torch.tensor([[0, 1, 2, -1, -1, -1, -1, -1, -1, -1]] * 8, dtype=torch.int32)
+    got, rec_l = _shards_combined(t, dev(t, cuda_device), 4)
+    assert torch.isinf(rec_l[3]).all()
+    ref = oracle_lib.forward(t.q, t.k_cache, t.v_cache, t.slot_idx, None, 1.0 / 16.0, block=4)
+    check_gates(got.float(), torch.from_numpy(ref), None, "context parallel empty shard")

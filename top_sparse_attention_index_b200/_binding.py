@@ -42,6 +42,11 @@ SIGNATURES = {
     "qsa_sparse_prefill_fp8kv": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64,
                                         _p, _i32, _i32, _i32, _i32, _i64, _i32, _i32, _f, _f, _f,
                                         _p, _i64, _i64, _i32, _p, _sz, _p, _p]),
+    "qsa_sparse_prefill_partial": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
+                                          _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _i32,
+                                          _i64, _i64, _i32, _f, _f, _f, _p, _p, _i32, _p, _sz, _p,
+                                          _p]),
+    "qsa_combine_partials": (_i32, [_p, _p, _i32, _i32, _i32, _i32, _p, _i64, _i64, _p]),
     "qsa_sparse_prefill_noalloc": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _f, _p,
                                           _i64, _i64, _i32, _p, _p]),
@@ -148,6 +153,26 @@ def qsa_sparse_prefill_fp8kv(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_s
         out_stride_t, out_stride_h, nsplit, workspace, workspace_bytes, err_word, stream))
 
 
+def qsa_sparse_prefill_partial(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
+                               v_cache, v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq,
+                               Hq, Hkv, D, S, W, block, slot_lo, S_total, kv_fp8, scale, k_scale,
+                               v_scale, part_o, part_lse, nsplit, workspace, workspace_bytes,
+                               err_word, stream) -> int:
+    """Raw call of one slot-range shard's partial record (context parallelism)."""
+    return int(load_library().qsa_sparse_prefill_partial(
+        q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache, v_stride_s,
+        v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W, block, slot_lo, S_total,
+        kv_fp8, ctypes.c_float(scale), ctypes.c_float(k_scale), ctypes.c_float(v_scale), part_o,
+        part_lse, nsplit, workspace, workspace_bytes, err_word, stream))
+
+
+def qsa_combine_partials(part_o, part_lse, R, Tq, Hq, D, out, out_stride_t, out_stride_h,
+                         stream) -> int:
+    """Raw call of the log-sum-exp combine of R stacked partial records."""
+    return int(load_library().qsa_combine_partials(part_o, part_lse, R, Tq, Hq, D, out,
+                                                   out_stride_t, out_stride_h, stream))
+
+
 def qsa_sparse_prefill_noalloc(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
                                v_cache, v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq,
                                Hq, Hkv, D, S, W, scale, out, out_stride_t, out_stride_h, nsplit,
@@ -229,6 +254,88 @@ def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=No
             st = qsa_sparse_prefill_fp8kv(*head, float(k_scale), float(v_scale), *tail)
         else:
             st = qsa_sparse_prefill_block(*head, *tail)
+    if st != QSA_OK:
+        raise QSAError(st, qsa_last_error_detail())
+    return out
+
+
+def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, width=None,
+                           scale=None, part_o=None, part_lse=None, nsplit=0, err_word=None,
+                           stream=None, block=1, k_scale=1.0, v_scale=1.0):
+    """One device's partial record for a cache split by slot range (context parallel).
+
+    k_cache / v_cache hold the global slots [slot_lo, slot_lo + S) of a cache of S_total
+    slots (bf16, or float8_e4m3fn codes with k_scale / v_scale); slot_idx holds global
+    slot numbers.  Returns (part_o fp32 [Tq, Hq, 256], part_lse fp32 [Tq, Hq]): the output
+    normalised over this device's valid slots and the base-2 log-sum-exp of their scaled
+    scores (-inf where there are none).  Combine the records of all devices with
+    combine_partials.
+    """
+    device = q.device
+    if device.type != "cuda":
+        raise ValueError("sparse_prefill_partial runs on CUDA tensors only")
+    Tq, Hq, D = q.shape
+    S, Hkv, Dk = k_cache.shape
+    if Dk != D or tuple(v_cache.shape) != (S, Hkv, D):
+        raise ValueError("k_cache and v_cache must both be [S, Hkv, D]")
+    if slot_idx.dim() != 2 or slot_idx.shape[0] != Tq:
+        raise ValueError("slot_idx must be [Tq, W]")
+    W = slot_idx.shape[1]
+    kv_fp8 = k_cache.dtype == torch.float8_e4m3fn
+    kv_dt = torch.float8_e4m3fn if kv_fp8 else torch.bfloat16
+    for name, t, dt in (("q", q, torch.bfloat16), ("k_cache", k_cache, kv_dt),
+                        ("v_cache", v_cache, kv_dt), ("slot_idx", slot_idx, torch.int32)):
+        _check_dev(name, t, dt, device)
+    if width is not None:
+        _check_dev("width", width, torch.int32, device)
+    if part_o is None:
+        part_o = torch.empty(Tq, Hq, D, dtype=torch.float32, device=device)
+    if part_lse is None:
+        part_lse = torch.empty(Tq, Hq, dtype=torch.float32, device=device)
+    for name, t, shape in (("part_o", part_o, (Tq, Hq, D)), ("part_lse", part_lse, (Tq, Hq))):
+        if tuple(t.shape) != shape or t.dtype != torch.float32 or not t.is_contiguous() or t.device != device:
+            raise ValueError(f"{name} must be a contiguous float32 {shape} tensor on {device}")
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    num_sms = torch.cuda.get_device_properties(device).multi_processor_count
+    ns, ws_bytes = qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, block, num_sms, nsplit)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device) if ws_bytes else None
+    with torch.cuda.device(device):
+        st = qsa_sparse_prefill_partial(
+            _ptr(q), q.stride(0), q.stride(1), _ptr(k_cache), k_cache.stride(0), k_cache.stride(1),
+            _ptr(v_cache), v_cache.stride(0), v_cache.stride(1), _ptr(slot_idx) if W else None,
+            slot_idx.stride(0), _ptr(width), Tq, Hq, Hkv, D, S, W, block, int(slot_lo),
+            int(S_total), 1 if kv_fp8 else 0, float(scale), float(k_scale), float(v_scale),
+            _ptr(part_o), _ptr(part_lse), ns, _ptr(ws), ws_bytes, _ptr(err_word),
+            stream.cuda_stream)
+    if st != QSA_OK:
+        raise QSAError(st, qsa_last_error_detail())
+    return part_o, part_lse
+
+
+def combine_partials(part_o, part_lse, out=None, stream=None):
+    """bf16 [Tq, Hq, 256]: the log-sum-exp combine of R stacked partial records
+    (part_o fp32 [R, Tq, Hq, 256], part_lse fp32 [R, Tq, Hq], both contiguous)."""
+    device = part_o.device
+    if device.type != "cuda":
+        raise ValueError("combine_partials runs on CUDA tensors only")
+    if part_o.dim() != 4 or part_lse.shape != part_o.shape[:3]:
+        raise ValueError("part_o must be [R, Tq, Hq, D] and part_lse [R, Tq, Hq]")
+    R, Tq, Hq, D = part_o.shape
+    for name, t in (("part_o", part_o), ("part_lse", part_lse)):
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.device != device:
+            raise ValueError(f"{name} must be a contiguous float32 tensor on {device}")
+    if out is None:
+        out = torch.empty(Tq, Hq, D, dtype=torch.bfloat16, device=device)
+    else:
+        _check_dev("out", out, torch.bfloat16, device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        st = qsa_combine_partials(_ptr(part_o), _ptr(part_lse), R, Tq, Hq, D, _ptr(out),
+                                  out.stride(0), out.stride(1), stream.cuda_stream)
     if st != QSA_OK:
         raise QSAError(st, qsa_last_error_detail())
     return out

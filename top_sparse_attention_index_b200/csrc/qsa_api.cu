@@ -153,6 +153,14 @@ int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, 
 
 namespace {
 
+// Slot-range shard and partial output of prefill_impl (context parallel).
+struct PartialArgs {
+  int64_t slot_lo = 0;
+  int64_t S_total = -1;  // -1: S (unsharded)
+  float* part_o = nullptr;
+  float* part_lse = nullptr;  // both set: write one normalised fp32 record + base-2 LSE
+};
+
 // The body shared by every launching entry point.  kv_fp8: k_cache / v_cache hold E4M3
 // codes (one byte per element, strides multiples of 16) dequantised with k_scale and
 // v_scale; otherwise bf16 (strides multiples of 8 elements) and the scales are 1.
@@ -164,7 +172,7 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
                           int32_t block, float scale, bool kv_fp8, float k_scale, float v_scale,
                           void* out, int64_t out_stride_t, int64_t out_stride_h, int32_t nsplit,
                           void* workspace, size_t workspace_bytes, uint32_t* err_word,
-                          void* stream) {
+                          void* stream, const PartialArgs& part = PartialArgs()) {
   g_detail[0] = '\0';
   qsa_status_t st = check_shape(Tq, Hq, Hkv, D, W);
   if (st == QSA_OK) st = check_block(block);
@@ -174,10 +182,27 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
   if (!std::isfinite(scale)) return fail(QSA_ERR_INVALID_ARG, "scale is not finite");
   if (!std::isfinite(k_scale) || !std::isfinite(v_scale))
     return fail(QSA_ERR_INVALID_ARG, "k_scale or v_scale is not finite");
+  const bool partial = part.part_o != nullptr || part.part_lse != nullptr;
+  const int64_t S_total = part.S_total < 0 ? S : part.S_total;
+  if (part.slot_lo < 0 || (S > 0 && part.slot_lo % block != 0))
+    return fail(QSA_ERR_INVALID_ARG, "slot_lo %lld must be a non-negative multiple of block %d",
+                (long long)part.slot_lo, block);
+  if (S_total < part.slot_lo + S)
+    return fail(QSA_ERR_INVALID_ARG, "S_total %lld below slot_lo + S = %lld", (long long)S_total,
+                (long long)(part.slot_lo + S));
+  if (S_total > int64_t(INT32_MAX) * block)
+    return fail(QSA_ERR_UNSUPPORTED, "S_total beyond the int32 selection range");
   if (Tq == 0) return QSA_OK;
 
-  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr)
+  // (an empty shard, S == 0, reads no cache row and may pass NULL caches)
+  if (q == nullptr || (S > 0 && (k_cache == nullptr || v_cache == nullptr)) ||
+      (!partial && out == nullptr))
     return fail(QSA_ERR_INVALID_ARG, "NULL q, k_cache, v_cache or out");
+  if (partial && (part.part_o == nullptr || part.part_lse == nullptr))
+    return fail(QSA_ERR_INVALID_ARG, "NULL part_o or part_lse");
+  if (partial && (!aligned16(part.part_o) || !aligned4(part.part_lse)))
+    return fail(QSA_ERR_INVALID_ARG, "part_o must be 16-byte and part_lse 4-byte aligned");
+  if (partial) out = part.part_o;  // (unused by the kernels in partial mode; keeps the checks)
   if (W > 0 && slot_idx == nullptr) return fail(QSA_ERR_INVALID_ARG, "NULL slot_idx with W > 0");
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
     return fail(QSA_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
@@ -255,6 +280,17 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
   p.kv_fp8 = kv_fp8 ? 1 : 0;
   p.v_scale = kv_fp8 ? v_scale : 1.0f;
   p.head_major = qsa::kernel_order_head_major(S, Hkv, int32_t(kv_elem));
+  p.slot_lo = part.slot_lo;
+  p.S_total = S_total;
+  if (partial) {
+    p.partial_out = 1;
+    p.part_o = part.part_o;
+    p.part_lse = part.part_lse;
+    if (pl.nsplit == 1) {  // the single split's record is the partial record itself
+      p.ws_o = part.part_o;
+      p.ws_lse = part.part_lse;
+    }
+  }
 
   const cudaError_t e = qsa::launch_sparse_prefill(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
@@ -278,6 +314,64 @@ qsa_status_t qsa_sparse_prefill_block(const void* q, int64_t q_stride_t, int64_t
                       v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W,
                       block, scale, false, 1.0f, 1.0f, out, out_stride_t, out_stride_h, nsplit,
                       workspace, workspace_bytes, err_word, stream);
+}
+
+qsa_status_t qsa_sparse_prefill_partial(const void* q, int64_t q_stride_t, int64_t q_stride_h,
+                                        const void* k_cache, int64_t k_stride_s,
+                                        int64_t k_stride_h, const void* v_cache,
+                                        int64_t v_stride_s, int64_t v_stride_h,
+                                        const int32_t* slot_idx, int64_t idx_stride_t,
+                                        const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
+                                        int32_t D, int64_t S, int32_t W, int32_t block,
+                                        int64_t slot_lo, int64_t S_total, int32_t kv_fp8,
+                                        float scale, float k_scale, float v_scale, float* part_o,
+                                        float* part_lse, int32_t nsplit, void* workspace,
+                                        size_t workspace_bytes, uint32_t* err_word, void* stream) {
+  if (kv_fp8 != 0 && kv_fp8 != 1) return fail(QSA_ERR_INVALID_ARG, "kv_fp8 must be 0 or 1");
+  PartialArgs part;
+  part.slot_lo = slot_lo;
+  part.S_total = S_total;
+  part.part_o = part_o;
+  part.part_lse = part_lse;
+  if (Tq > 0 && (part_o == nullptr || part_lse == nullptr)) {
+    g_detail[0] = '\0';
+    return fail(QSA_ERR_INVALID_ARG, "NULL part_o or part_lse");
+  }
+  if (S_total < 0) return fail(QSA_ERR_INVALID_ARG, "negative S_total");
+  return prefill_impl(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,
+                      v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W,
+                      block, scale, kv_fp8 != 0, kv_fp8 ? k_scale : 1.0f, kv_fp8 ? v_scale : 1.0f,
+                      nullptr, 0, 0, nsplit, workspace, workspace_bytes, err_word, stream, part);
+}
+
+qsa_status_t qsa_combine_partials(const float* part_o, const float* part_lse, int32_t R,
+                                  int32_t Tq, int32_t Hq, int32_t D, void* out,
+                                  int64_t out_stride_t, int64_t out_stride_h, void* stream) {
+  g_detail[0] = '\0';
+  if (R < 1 || Tq < 0 || Hq < 1)
+    return fail(QSA_ERR_INVALID_ARG, "bad sizes: R=%d Tq=%d Hq=%d", R, Tq, Hq);
+  if (D != qsa::kHeadDim) return fail(QSA_ERR_UNSUPPORTED, "head dimension %d (only 256)", D);
+  if (Tq == 0) return QSA_OK;
+  if (part_o == nullptr || part_lse == nullptr || out == nullptr)
+    return fail(QSA_ERR_INVALID_ARG, "NULL part_o, part_lse or out");
+  if (!aligned16(part_o) || !aligned4(part_lse) || !aligned16(out))
+    return fail(QSA_ERR_INVALID_ARG, "part_o and out must be 16-byte, part_lse 4-byte aligned");
+  if (!stride_ok(out_stride_t) || !stride_ok(out_stride_h))
+    return fail(QSA_ERR_INVALID_ARG, "out strides must be non-negative multiples of 8 elements");
+  if (int64_t(Tq) * Hq > int64_t(INT32_MAX) * 4)
+    return fail(QSA_ERR_INVALID_ARG, "too many rows for one launch");
+  qsa::FwdParams p{};
+  p.ws_o = const_cast<float*>(part_o);
+  p.ws_lse = const_cast<float*>(part_lse);
+  p.out = static_cast<uint16_t*>(out);
+  p.out_stride_t = out_stride_t;
+  p.out_stride_h = out_stride_h;
+  p.Tq = Tq;
+  p.Hq = Hq;
+  p.nsplit = R;
+  const cudaError_t e = qsa::launch_combine(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e));
+  return QSA_OK;
 }
 
 qsa_status_t qsa_sparse_prefill_fp8kv(const void* q, int64_t q_stride_t, int64_t q_stride_h,

@@ -159,15 +159,19 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   const int per = (n_raw + C::kThreads - 1) / C::kThreads;
   const int b_i = min(tid * per, n_raw);
   const int e_i = min(b_i + per, n_raw);
-  // An entry is valid when its whole block of p.block slots lies in [0, S).
+  // An entry is valid when its whole block of p.block slots lies in [0, S_total); it is
+  // local when that block lies in this cache's range [slot_lo, slot_lo + S).
   const int block = p.block;
+  const int64_t lo = p.slot_lo, hi = p.slot_lo + p.S;
+  auto local = [&](int v) {
+    return v >= 0 && int64_t(v) * block >= lo && (int64_t(v) + 1) * block <= hi;
+  };
   int cnt = 0;
   bool bad = false;
   for (int i = b_i; i < e_i; ++i) {
     const int v = sRaw[i];
-    const bool ok = v >= 0 && (int64_t(v) + 1) * block <= p.S;
-    bad |= (!ok && v != -1);
-    cnt += ok ? block : 0;
+    bad |= v != -1 && !(v >= 0 && (int64_t(v) + 1) * block <= p.S_total);
+    cnt += local(v) ? block : 0;
   }
   if (bad && p.err_word != nullptr) atomicOr(p.err_word, 1u);
   int incl = cnt;
@@ -189,9 +193,9 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     int pos = warp_off + incl - cnt;
     for (int i = b_i; i < e_i; ++i) {
       const int v = sRaw[i];
-      if (v >= 0 && (int64_t(v) + 1) * block <= p.S) {
+      if (local(v)) {
         for (int e = 0; e < block; ++e) {
-          const uint32_t slot = uint32_t(v) * uint32_t(block) + uint32_t(e);
+          const uint32_t slot = uint32_t(int64_t(v) * block + e - lo);  // row of this cache
           sSlot[pos++] = slot;
         }
       }
@@ -202,7 +206,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   const int G = p.G;
   const int64_t head0 = int64_t(j) * G;
   if (n_valid == 0) {  // fully masked row, zero width or an empty split (block-uniform)
-    if (p.nsplit == 1) {
+    if (p.nsplit == 1 && !p.partial_out) {
       for (int i = tid; i < G * kChunks; i += C::kThreads) {
         const int g = i / kChunks, c = i % kChunks;
         uint16_t* dst = p.out + int64_t(t) * p.out_stride_t + (head0 + g) * p.out_stride_h + c * 8;
@@ -211,6 +215,13 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     } else {
       for (int g = tid; g < G; g += C::kThreads)
         p.ws_lse[(int64_t(split) * p.Tq + t) * p.Hq + head0 + g] = kNegInf;
+      if (p.nsplit == 1) {  // a partial record (the combine skips it): O written as zeros
+        for (int i = tid; i < G * (kHeadDim / 4); i += C::kThreads) {
+          const int g = i / (kHeadDim / 4), c = i % (kHeadDim / 4);
+          reinterpret_cast<float4*>(p.ws_o + (int64_t(t) * p.Hq + head0 + g) * kHeadDim)[c] =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
     }
     return;
   }
@@ -645,7 +656,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     }
     const float inv = (KV8 ? p.v_scale : 1.f) / lsum;
     const int64_t h = head0 + gg;
-    if (p.nsplit == 1) {
+    if (p.nsplit == 1 && !p.partial_out) {
       uint4 v;
       v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
       v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
@@ -671,9 +682,15 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
   float mstar = kNegInf;
   for (int s = 0; s < p.nsplit; ++s) mstar = fmaxf(mstar, p.ws_lse[s * rows + row]);
   const int64_t t = row / p.Hq, h = row % p.Hq;
-  uint4* dst = reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8);
-  if (mstar == kNegInf) {
-    *dst = make_uint4(0u, 0u, 0u, 0u);
+  if (mstar == kNegInf) {  // no valid slot in any split
+    if (p.partial_out) {
+      float4* po = reinterpret_cast<float4*>(p.part_o + row * kHeadDim + lane * 8);
+      po[0] = po[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (lane == 0) p.part_lse[row] = kNegInf;
+    } else {
+      *reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
     return;
   }
   float acc[8];
@@ -691,12 +708,19 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
     acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
   }
   const float inv = 1.f / wsum;
+  if (p.partial_out) {  // one normalised record of all splits: O and lse* + log2(sum of weights)
+    float4* po = reinterpret_cast<float4*>(p.part_o + row * kHeadDim + lane * 8);
+    po[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    po[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+    if (lane == 0) p.part_lse[row] = mstar + fast_log2(wsum);
+    return;
+  }
   uint4 v;
   v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
   v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
   v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  *dst = v;
+  *reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8) = v;
 }
 
 template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8>
@@ -813,7 +837,12 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
                                 kLargeQsplit, false>(p, stream);
   }
   if (e != cudaSuccess || p.nsplit == 1) return e;
+  return launch_combine(p, stream);
+}
+
+cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream) {
   const int64_t rows = int64_t(p.Tq) * p.Hq;
+  if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
   qsa_lse_combine_kernel<<<grid, 128, 0, stream>>>(p);
   return cudaGetLastError();

@@ -45,6 +45,16 @@ struct FwdParams {
   int32_t kv_fp8;           // 1: k_cache / v_cache hold E4M3 codes
   float v_scale;            // E4M3 cache: multiplier of the normalised output
   int32_t head_major;       // 1: work units ordered KV head slowest (see kernel_order)
+  // Slot-range shard (context parallel): k_cache / v_cache hold global slots
+  // [slot_lo, slot_lo + S); selected slots elsewhere in [0, S_total) are not local (not
+  // an error); S_total = S and slot_lo = 0 for an unsharded call.
+  int64_t slot_lo;
+  int64_t S_total;
+  // 1: write the normalised fp32 O and the base-2 LSE (ws_o / ws_lse layout, the call's
+  // own split plan combined into one record per (t, h)) instead of bf16 out
+  int32_t partial_out;
+  float* part_o;            // partial_out: fp32 [Tq, Hq, D]
+  float* part_lse;          // partial_out: fp32 [Tq, Hq]
 };
 
 // Kernel configuration chosen for a group size G (shared by planner and launcher).
@@ -72,6 +82,10 @@ inline int32_t kernel_order_head_major(int64_t S, int32_t Hkv, int32_t kv_elem_b
 
 // Enqueue the fused kernel (and the combine when nsplit > 1) on `stream`.
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream);
+
+// Enqueue the LSE combine of p.nsplit partial records (p.ws_o / p.ws_lse) into bf16 out,
+// or into one partial record (p.part_o / p.part_lse) when p.partial_out.
+cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream);
 
 size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit);
 

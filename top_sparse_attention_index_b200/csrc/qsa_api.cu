@@ -280,8 +280,9 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
   p.kv_fp8 = kv_fp8 ? 1 : 0;
   p.v_scale = kv_fp8 ? v_scale : 1.0f;
   p.head_major = qsa::kernel_order_head_major(S, Hkv, int32_t(kv_elem));
-  p.slot_lo = part.slot_lo;
-  p.S_total = S_total;
+  p.ent_lo = int32_t(part.slot_lo / block);
+  p.ent_hi = int32_t((part.slot_lo + S) / block);
+  p.ent_total = int32_t(S_total / block);
   if (partial) {
     p.partial_out = 1;
     p.part_o = part.part_o;

@@ -159,18 +159,17 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   const int per = (n_raw + C::kThreads - 1) / C::kThreads;
   const int b_i = min(tid * per, n_raw);
   const int e_i = min(b_i + per, n_raw);
-  // An entry is valid when its whole block of p.block slots lies in [0, S_total); it is
-  // local when that block lies in this cache's range [slot_lo, slot_lo + S).
+  // An entry is valid when its whole block of p.block slots lies in the cache's global
+  // extent (0 <= v < ent_total) and local when that block is held here (ent_lo <= v <
+  // ent_hi); unsigned compares cover the negative values.
   const int block = p.block;
-  const int64_t lo = p.slot_lo, hi = p.slot_lo + p.S;
-  auto local = [&](int v) {
-    return v >= 0 && int64_t(v) * block >= lo && (int64_t(v) + 1) * block <= hi;
-  };
+  const uint32_t ent_lo = uint32_t(p.ent_lo), ent_n = uint32_t(p.ent_hi - p.ent_lo);
+  auto local = [&](int v) { return uint32_t(v) - ent_lo < ent_n; };
   int cnt = 0;
   bool bad = false;
   for (int i = b_i; i < e_i; ++i) {
     const int v = sRaw[i];
-    bad |= v != -1 && !(v >= 0 && (int64_t(v) + 1) * block <= p.S_total);
+    bad |= v != -1 && uint32_t(v) >= uint32_t(p.ent_total);
     cnt += local(v) ? block : 0;
   }
   if (bad && p.err_word != nullptr) atomicOr(p.err_word, 1u);
@@ -194,10 +193,8 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     for (int i = b_i; i < e_i; ++i) {
       const int v = sRaw[i];
       if (local(v)) {
-        for (int e = 0; e < block; ++e) {
-          const uint32_t slot = uint32_t(int64_t(v) * block + e - lo);  // row of this cache
-          sSlot[pos++] = slot;
-        }
+        const uint32_t row = (uint32_t(v) - ent_lo) * uint32_t(block);  // row of this cache
+        for (int e = 0; e < block; ++e) sSlot[pos++] = row + uint32_t(e);
       }
     }
   }

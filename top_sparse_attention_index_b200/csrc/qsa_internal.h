@@ -45,11 +45,14 @@ struct FwdParams {
   int32_t kv_fp8;           // 1: k_cache / v_cache hold E4M3 codes
   float v_scale;            // E4M3 cache: multiplier of the normalised output
   int32_t head_major;       // 1: work units ordered KV head slowest (see kernel_order)
-  // Slot-range shard (context parallel): k_cache / v_cache hold global slots
-  // [slot_lo, slot_lo + S); selected slots elsewhere in [0, S_total) are not local (not
-  // an error); S_total = S and slot_lo = 0 for an unsharded call.
-  int64_t slot_lo;
-  int64_t S_total;
+  // Selected entries (slot numbers, or block numbers with block selection): an entry v is
+  // valid when 0 <= v < ent_total and local when ent_lo <= v < ent_hi; the cache holds the
+  // rows of the local entries, row (v - ent_lo) * block + e.  Unsharded: ent_lo = 0,
+  // ent_hi = ent_total = floor(S / block); a slot-range shard [slot_lo, slot_lo + S) of a
+  // cache of S_total slots: slot_lo / block, floor((slot_lo + S) / block), S_total / block.
+  int32_t ent_lo;
+  int32_t ent_hi;
+  int32_t ent_total;
   // 1: write the normalised fp32 O and the base-2 LSE (ws_o / ws_lse layout, the call's
   // own split plan combined into one record per (t, h)) instead of bf16 out
   int32_t partial_out;

@@ -590,3 +590,33 @@ def test_context_parallel_block4_and_empty_shard(cuda_device, oracle_lib):
     assert torch.isinf(rec_l[3]).all()
     ref = oracle_lib.forward(t.q, t.k_cache, t.v_cache, t.slot_idx, None, 1.0 / 16.0, block=4)
     check_gates(got.float(), torch.from_numpy(ref), None, "context parallel empty shard")
+
+
+def test_context_parallel_nccl_world_of_one(cuda_device):
+    """The public context-parallel call end to end on one GPU: a one-rank NCCL group,
+    its all-gather and the combine; one shard holding the whole cache gives bitwise the
+    unsharded call."""
+    import datetime
+    import os
+    import socket
+
+    import torch.distributed as dist
+    if dist.is_initialized():
+        pytest.skip("a process group already exists")
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=cuda_device,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = _random_case(89, 200, 16, 2, 16384, 2051, minus1=0.05, widths=True)
+        d = dev(w, cuda_device)
+        lo, hi = qsa.shard_ranges(w.S, dist.get_world_size())[dist.get_rank()]
+        out = qsa.sparse_prefill_context_parallel(d["q"], d["k_cache"][lo:hi], d["v_cache"][lo:hi],
+                                                  d["slot_idx"], lo, w.S, width=d["width"])
+        torch.cuda.synchronize()
+        assert torch.equal(out.cpu().view(torch.int16), run(d, 1.0 / 16.0).view(torch.int16))
+    finally:
+        dist.destroy_process_group()

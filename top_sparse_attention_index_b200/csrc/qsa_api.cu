@@ -202,9 +202,9 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
     return fail(QSA_ERR_INVALID_ARG, "NULL part_o or part_lse");
   if (partial && (!aligned16(part.part_o) || !aligned4(part.part_lse)))
     return fail(QSA_ERR_INVALID_ARG, "part_o must be 16-byte and part_lse 4-byte aligned");
-  if (partial) out = part.part_o;  // (unused by the kernels in partial mode; keeps the checks)
   if (W > 0 && slot_idx == nullptr) return fail(QSA_ERR_INVALID_ARG, "NULL slot_idx with W > 0");
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+  // (in partial mode `out` is not used: the record buffers take its place)
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || (!partial && !aligned16(out)))
     return fail(QSA_ERR_INVALID_ARG, "q, k_cache, v_cache and out must be 16-byte aligned");
   if ((slot_idx != nullptr && !aligned4(slot_idx)) || (width != nullptr && !aligned4(width)) ||
       (err_word != nullptr && !aligned4(err_word)))

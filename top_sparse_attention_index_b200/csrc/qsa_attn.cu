@@ -146,6 +146,20 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     }
     width_t = wv;
   }
+  // ---- 0. the group's Q rows (commit group 0): in flight during the index work ---------
+  const int G = p.G;
+  const int64_t head0 = int64_t(j) * G;
+  const uint32_t ring_s = smem_addr(ring);
+  const uint32_t q_s = smem_addr(sQ);
+  for (int i = tid; i < NTILE * 8 * kChunks; i += C::kThreads) {
+    const int g = i / kChunks, c = i % kChunks;
+    const bool ok = g < G;
+    const uint16_t* src =
+        p.q + int64_t(t) * p.q_stride_t + (head0 + (ok ? g : 0)) * p.q_stride_h + c * 8;
+    cp_async_16(q_s + g * kRowBytes + ((c ^ (g & 7)) << 4), src, ok);
+  }
+  cp_async_commit();
+
   const int w0 = split * p.split_len;
   const int n_raw = max(min(w0 + p.split_len, width_t) - w0, 0);
 
@@ -200,9 +214,8 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   }
   __syncthreads();  // sSlot complete, the ring is free again
 
-  const int G = p.G;
-  const int64_t head0 = int64_t(j) * G;
   if (n_valid == 0) {  // fully masked row, zero width or an empty split (block-uniform)
+    cp_async_wait<0>();  // the Q copy lands before this CTA's shared memory is released
     if (p.nsplit == 1 && !p.partial_out) {
       for (int i = tid; i < G * kChunks; i += C::kThreads) {
         const int g = i / kChunks, c = i % kChunks;
@@ -223,17 +236,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     return;
   }
 
-  // ---- 2. Q tile (group 0) and the pipeline prologue ------------------------------------
-  const uint32_t ring_s = smem_addr(ring);
-  const uint32_t q_s = smem_addr(sQ);
-  for (int i = tid; i < NTILE * 8 * kChunks; i += C::kThreads) {
-    const int g = i / kChunks, c = i % kChunks;
-    const bool ok = g < G;
-    const uint16_t* src =
-        p.q + int64_t(t) * p.q_stride_t + (head0 + (ok ? g : 0)) * p.q_stride_h + c * 8;
-    cp_async_16(q_s + g * kRowBytes + ((c ^ (g & 7)) << 4), src, ok);
-  }
-  cp_async_commit();
+  // ---- 2. the pipeline prologue -------------------------------------------------------
 
   const int n_stages = (n_valid + C::kRows - 1) / C::kRows;
   // Pad the offset list to whole 16-slot sub-tiles with the first slot: padding rows

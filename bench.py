@@ -56,7 +56,7 @@ L2_FLUSH_BYTES = 512 << 20
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
@@ -333,6 +333,19 @@ def main():
     total_ms = reduce_max(sum(kernel_ms), dist, device)   # the slowest rank's device time
     ms_per_step = total_ms / args.steps
 
+    # warm-cache figure, outside the timed region: the same launch repeated with no L2
+    # flush in between, median over the launches (the slowest rank's median)
+    n_warm = min(args.steps, 50)
+    w_starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_warm)]
+    w_ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_warm)]
+    for i in range(n_warm):
+        w_starts[i].record(stream)
+        step()
+        w_ends[i].record(stream)
+    torch.cuda.synchronize()
+    warm_ms = reduce_max(statistics.median(s.elapsed_time(e) for s, e in zip(w_starts, w_ends)),
+                         dist, device)
+
     # end to end through the public host-buffer API: pinned host inputs -> device ->
     # kernels -> pinned host output, transfers overlapped with the kernels by row chunks
     e2e = None
@@ -405,6 +418,9 @@ def main():
         # the bound that binds once the gathered rows are L2 hits: every gathered byte
         # is written to shared memory once (cp.async) and read once (ldmatrix)
         "shared_memory": _smem_bound(gathered, t_s, clocks.summary(t0_epoch, t1_epoch)),
+        "warm_l2": {"ms_per_step_median": warm_ms, "launches": n_warm,
+                    "value": world * flops / (warm_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "note": "no L2 flush between launches; not the timed region"},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clocks.summary(t0_epoch, t1_epoch),
         "wall_s_timed_region": t_wall,

@@ -458,6 +458,19 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     for (int nt = 0; nt < TPW; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc[nt][e] = sa[nt][e] + sb[nt][e];
+    // With one head tile per warp the first kVEarly V fragments of the sub-tile (bf16: m-tiles;
+    // E4M3: raw codes of m-tile pairs) are read here, before the score exchange and the
+    // softmax, so their shared-memory latency is hidden behind that work (the stage has
+    // landed; the registers fit under the two-CTA cap).  With two head tiles per warp the
+    // registers are already at the cap and the early reads cost more than they hide.
+    constexpr int kVEarly = TPW == 1 ? (KV8 ? 2 : 4) : 0;
+    uint32_t vt[4];
+    uint32_t vearly[kVEarly > 0 ? kVEarly : 1][4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / (KV8 ? 8 : 4)) * 128;
+#pragma unroll
+    for (int mt = 0; mt < kVEarly; ++mt)
+      ldmatrix_x4_trans(vearly[mt], vt[mt & 3] + 128 * (mt >> 2));
     if constexpr (QSPLIT) {
       // each warp of the pair holds the scores over its half of D: exchange and add in
       // a fixed order (low half + high half) so both warps hold the same scores
@@ -552,14 +565,15 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
 
     // O^T (this warp's D rows x 8) += V^T (D rows x 16) * P^T (16 x 8) per head tile;
     // each V fragment feeds every tile of the warp
-    uint32_t vt[4];
     if constexpr (!KV8) {
-#pragma unroll
-      for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / 4) * 128;
 #pragma unroll
       for (int mt = 0; mt < kMT; ++mt) {
         uint32_t a[4];
-        ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
+        if (mt < kVEarly) {
+          a[0] = vearly[mt][0]; a[1] = vearly[mt][1]; a[2] = vearly[mt][2]; a[3] = vearly[mt][3];
+        } else {
+          ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
+        }
 #pragma unroll
         for (int nt = 0; nt < TPW; ++nt) mma_bf16_16816(o[nt][mt], a, b0[nt], b1[nt]);
       }
@@ -569,11 +583,13 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
       // the two slots of each d, so tile row l/4 is d = 16 c + 2(l/4) and row l/4 + 8
       // is d + 1.  r0 / r1: slots 0-7 / 8-15 of chunk 2 mq, r2 / r3 of chunk 2 mq + 1.
 #pragma unroll
-      for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / 8) * 128;
-#pragma unroll
       for (int mq = 0; mq < kMT / 2; ++mq) {
         uint32_t r[4], a[4];
-        ldmatrix_x4_trans(r, vt[mq & 3] + 128 * (mq >> 2));
+        if (mq < kVEarly) {
+          r[0] = vearly[mq][0]; r[1] = vearly[mq][1]; r[2] = vearly[mq][2]; r[3] = vearly[mq][3];
+        } else {
+          ldmatrix_x4_trans(r, vt[mq & 3] + 128 * (mq >> 2));
+        }
         e4m3x4_to_f16x2x2(byte_perm(r[0], 0u, 0x3120u), a[0], a[1]);
         e4m3x4_to_f16x2x2(byte_perm(r[1], 0u, 0x3120u), a[2], a[3]);
 #pragma unroll

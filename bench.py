@@ -418,6 +418,8 @@ def main():
         # the bound that binds once the gathered rows are L2 hits: every gathered byte
         # is written to shared memory once (cp.async) and read once (ldmatrix)
         "shared_memory": _smem_bound(gathered, t_s, clocks.summary(t0_epoch, t1_epoch)),
+        # the bound of the L2-resident gather (most gathered rows are L2 hits)
+        "l2": _l2_bound(alg_bytes, t_s),
         "warm_l2": {"ms_per_step_median": warm_ms, "launches": n_warm,
                     "value": world * flops / (warm_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "note": "no L2 flush between launches; not the timed region"},
@@ -440,6 +442,22 @@ def _smem_bound(gathered: int, t_s: float, clk: dict, sms: int = 148) -> dict:
     achieved = 2 * gathered / t_s / 1e12
     return {"bytes_per_launch": 2 * gathered, "achieved": achieved, "peak": peak,
             "unit": "TB/s", "frac": achieved / peak, "sm_mhz": mhz}
+
+
+# L2 -> SM read peak of this B200, from the peak rates ncu reports for the kernel: 184 L2
+# slices (lts__cycles_elapsed.sum / .avg) x 2 sectors per slice clock
+# (lts__t_sectors_srcunit_tex peak_sustained) x 32 B x the 1.955 GHz L2 clock
+# (lts__cycles_elapsed.avg.per_second) = 23.0 TB/s
+L2_READ_PEAK_TBS = 184 * 2 * 32 * 1.955e9 / 1e12
+
+
+def _l2_bound(alg_bytes: int, t_s: float) -> dict:
+    """L2 read roofline: every algorithmic byte (gathered K/V rows, Q, indices) is read
+    from L2 by the SMs, hit or miss, against the ncu-derived L2 -> SM read peak."""
+    achieved = alg_bytes / t_s / 1e12
+    return {"bytes_per_launch": alg_bytes, "achieved": achieved, "peak": L2_READ_PEAK_TBS,
+            "unit": "TB/s", "frac": achieved / L2_READ_PEAK_TBS,
+            "peak_source": "ncu-derived: 184 L2 slices x 2 sectors/clk x 32 B x 1.955 GHz"}
 
 
 def _kernel_hash():

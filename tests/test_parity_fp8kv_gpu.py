@@ -286,3 +286,38 @@ def test_context_parallel_shards(cuda_device, oracle_lib):
     w = _random_case(2800, 200, 16, 2, 16384, 2051, minus1=0.05, widths=True)
     got, _ = _shards_combined(w, dev(w, cuda_device), 3, k_scale=w.k_scale, v_scale=w.v_scale)
     compare(w, got, oracle_lib, 1.0 / 16.0, None, "e4m3 context parallel R=3")
+
+
+def test_cache_offsets_beyond_4gib(cuda_device, oracle_lib):
+    """S = 18,000,000 slots at Hkv = 1: the E4M3 K and V caches are 4.6 GB each (256-byte
+    rows), and half of every row's selection lies past byte offset 4 GiB (slot
+    16,777,216), where a 32-bit row offset would wrap.  Only the selected rows hold
+    codes; the oracle runs on a compact copy with the indices renumbered."""
+    S, Hq, Hkv, Tq, W = 18_000_000, 8, 1, 48, 1500
+    far = S - (1 << 24)
+    g = torch.Generator().manual_seed(406)
+    a = (S - far) + wl.uniform_distinct(g, Tq, far, W // 2)
+    b = wl.uniform_distinct(g, Tq, S - far, W - W // 2)
+    idx = torch.cat([a, b], dim=1)
+    idx = torch.gather(idx, 1, torch.argsort(torch.rand(Tq, W, generator=g), dim=1)).to(torch.int32)
+    idx[:, ::11] = -1
+    used = torch.unique(idx[idx >= 0])
+    rows_k = wl.to_e4m3_cache(torch.randn(used.numel(), Hkv, D, generator=g), KS)
+    rows_v = wl.to_e4m3_cache(torch.randn(used.numel(), Hkv, D, generator=g), VS)
+    q = torch.randn(Tq, Hq, D, generator=g).to(torch.bfloat16)
+    k_dev = torch.zeros(S, Hkv, D, dtype=torch.uint8, device=cuda_device)
+    v_dev = torch.zeros(S, Hkv, D, dtype=torch.uint8, device=cuda_device)
+    k_dev[used.to(cuda_device)] = rows_k.view(torch.uint8).to(cuda_device)
+    v_dev[used.to(cuda_device)] = rows_v.view(torch.uint8).to(cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = qsa.sparse_prefill(q.to(cuda_device), k_dev.view(torch.float8_e4m3fn),
+                             v_dev.view(torch.float8_e4m3fn), idx.to(cuda_device), scale=1.0 / 16.0,
+                             k_scale=KS, v_scale=VS, err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    remap = torch.full((S,), -1, dtype=torch.int32)
+    remap[used] = torch.arange(used.numel(), dtype=torch.int32)
+    idx_c = torch.where(idx >= 0, remap[idx.clamp(min=0).long()], idx)
+    ref = oracle_lib.forward_fp8kv(q, rows_k, rows_v, idx_c, None, 1.0 / 16.0, KS, VS)
+    check_gates(out.cpu().float(), torch.from_numpy(ref), None, "E4M3 cache past 4 GiB")
+    del k_dev, v_dev

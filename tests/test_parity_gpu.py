@@ -490,6 +490,70 @@ def test_large_cache_two_million_slots(cuda_device, oracle_lib):
     del k_dev, v_dev
 
 
+def _far_and_near(g, Tq, S, W, far):
+    """Distinct slots per row: W // 2 from the last `far` slots of the cache, the rest
+    from below them (shuffled together)."""
+    a = (S - far) + wl.uniform_distinct(g, Tq, far, W // 2)
+    b = wl.uniform_distinct(g, Tq, S - far, W - W // 2)
+    idx = torch.cat([a, b], dim=1)
+    perm = torch.argsort(torch.rand(Tq, W, generator=g), dim=1)
+    return torch.gather(idx, 1, perm).to(torch.int32)
+
+
+def test_cache_offsets_beyond_4gib(cuda_device, oracle_lib):
+    """S = 9,000,000 slots at Hkv = 1: K and V are 4.6 GB each, and half of every row's
+    selection lies past byte offset 4 GiB (slot 8,388,608), where a 32-bit row offset
+    would wrap to another row.  Only the selected rows hold data; the oracle runs on a
+    compact copy with the indices renumbered."""
+    S, Hq, Hkv, Tq, W = 9_000_000, 8, 1, 48, 1500
+    g = torch.Generator().manual_seed(404)
+    idx = _far_and_near(g, Tq, S, W, far=S - (1 << 23))
+    assert int((idx >= (1 << 23)).sum()) >= Tq * (W // 2)
+    idx[:, ::11] = -1
+    used = torch.unique(idx[idx >= 0])
+    rows_k = torch.randn(used.numel(), Hkv, D, generator=g).to(torch.bfloat16)
+    rows_v = torch.randn(used.numel(), Hkv, D, generator=g).to(torch.bfloat16)
+    q = torch.randn(Tq, Hq, D, generator=g).to(torch.bfloat16)
+    k_dev = torch.zeros(S, Hkv, D, dtype=torch.bfloat16, device=cuda_device)
+    v_dev = torch.zeros(S, Hkv, D, dtype=torch.bfloat16, device=cuda_device)
+    k_dev[used.to(cuda_device)] = rows_k.to(cuda_device)
+    v_dev[used.to(cuda_device)] = rows_v.to(cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    out = qsa.sparse_prefill(q.to(cuda_device), k_dev, v_dev, idx.to(cuda_device), err_word=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    remap = torch.full((S,), -1, dtype=torch.int32)
+    remap[used] = torch.arange(used.numel(), dtype=torch.int32)
+    idx_c = torch.where(idx >= 0, remap[idx.clamp(min=0).long()], idx)
+    ref = oracle_lib.forward(q, rows_k, rows_v, idx_c, None, 1.0 / 16.0)
+    check_gates(out.cpu().float(), torch.from_numpy(ref), None, "cache past 4 GiB")
+    del k_dev, v_dev
+
+
+def test_query_and_output_offsets_beyond_2gib(cuda_device, oracle_lib):
+    """Tq = 270,000 rows at Hq = 16: Q and the output are 2.2 GB each, so rows from
+    262,144 on start past byte offset 2 GiB (a signed 32-bit offset would be negative).
+    Q repeats one 1,000-row block (built on the device by torch); the oracle checks the
+    first rows, rows around the 2 GiB boundary and the last rows."""
+    Tq, Hq, Hkv, S, W = 270_000, 16, 2, 4096, 8
+    g = torch.Generator().manual_seed(405)
+    q_small = torch.randn(1000, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(S, Hkv, D, generator=g).to(torch.bfloat16)
+    idx = wl.uniform_distinct(g, Tq, S, W)
+    idx[::5, 3] = -1
+    idx[Tq - 1] = -1  # the very last row is empty: exact zeros past 2 GiB
+    q_dev = q_small.to(cuda_device).repeat(Tq // 1000, 1, 1)
+    out = qsa.sparse_prefill(q_dev, k.to(cuda_device), v.to(cuda_device), idx.to(cuda_device))
+    torch.cuda.synchronize()
+    rows = (list(range(0, 8)) + list(range(262_140, 262_150)) + list(range(Tq - 9, Tq)))
+    got = out[torch.tensor(rows, device=cuda_device)].cpu()
+    r = torch.tensor(rows)
+    ref = oracle_lib.forward(q_small[r % 1000], k, v, idx[r], None, 1.0 / 16.0)
+    check_gates(got.float(), torch.from_numpy(ref), [len(rows) - 1], "output past 2 GiB")
+    del q_dev, out
+
+
 def test_very_wide_selection(cuda_device, oracle_lib):
     """W = 20,000 selected slots per row: at least eight splits, combined by the LSE
     kernel."""

@@ -376,7 +376,9 @@ def sparse_prefill_from_host(q, k_cache, v_cache, slot_idx, width=None, scale=No
     if out is None:
         out = torch.empty(Tq, Hq, D, dtype=torch.bfloat16).pin_memory()
     if chunk_rows is None:
-        chunk_rows = max(-(-Tq // 16), 256)
+        # eight chunks: measured best for the long prefill (5.46 ms; 16 chunks 5.61, four
+        # 5.83; chunks shrinking towards the end were slower still)
+        chunk_rows = max(-(-Tq // 8), 256)
     if nsplit == 0:
         # every chunk uses the whole batch's split plan, so the result does not depend
         # on the chunking: it is bitwise that of one device call on the whole batch

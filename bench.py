@@ -415,11 +415,12 @@ def main():
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": alg_bytes},
-        # the bound that binds once the gathered rows are L2 hits: every gathered byte
-        # is written to shared memory once (cp.async) and read once (ldmatrix)
+        # the bounds that bind once the gathered rows are L2 hits: the rate at which
+        # shared memory takes the copied rows while they are read back, and the L2 ->
+        # shared-memory gather rate alone
         "shared_memory": _smem_bound(gathered, t_s, clocks.summary(t0_epoch, t1_epoch)),
         # the bound of the L2-resident gather (most gathered rows are L2 hits)
-        "l2": _l2_bound(alg_bytes, t_s),
+        "l2": _l2_bound(gathered, t_s, clocks.summary(t0_epoch, t1_epoch)),
         "warm_l2": {"ms_per_step_median": warm_ms, "launches": n_warm,
                     "value": world * flops / (warm_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "note": "no L2 flush between launches; not the timed region"},
@@ -434,30 +435,40 @@ def main():
     print(json.dumps(result))
 
 
+# Shared-memory and L2 rates of this B200, measured by a probe with the gather's access
+# pattern (one CTA of 16 warps per SM; cp.async.cg copies of random 512-byte rows of an
+# L2-resident 64 MB buffer into shared memory, ldmatrix.x4 reads of shared memory; cycles
+# by clock64):  fills alone 115.8 B per SM clock, ldmatrix reads alone 126.3; both at once
+# 84.1 B/clk of fills beside 98.5 of reads.
+GATHER_FILL_ALONE_B_PER_CLK = 115.8
+GATHER_FILL_WITH_READS_B_PER_CLK = 84.1
+
+
 def _smem_bound(gathered: int, t_s: float, clk: dict, sms: int = 148) -> dict:
-    """Shared-memory round-trip roofline: 2 x gathered bytes against sms x 128 B per
-    SM clock at the median SM clock sampled during the timed region."""
+    """Shared-memory bound of the gather: every gathered byte is copied into shared memory
+    (cp.async) and read back once (ldmatrix); with both streams equal, the fill rate
+    measured beside concurrent reads binds (sms x 84.1 B per SM clock at the median SM
+    clock sampled during the timed region)."""
     mhz = clk.get("sm_mhz") or 1965.0
-    peak = sms * 128 * mhz * 1e6 / 1e12
-    achieved = 2 * gathered / t_s / 1e12
-    return {"bytes_per_launch": 2 * gathered, "achieved": achieved, "peak": peak,
-            "unit": "TB/s", "frac": achieved / peak, "sm_mhz": mhz}
+    peak = sms * GATHER_FILL_WITH_READS_B_PER_CLK * mhz * 1e6 / 1e12
+    achieved = gathered / t_s / 1e12
+    return {"bytes_per_launch": gathered, "achieved": achieved, "peak": peak,
+            "unit": "TB/s", "frac": achieved / peak, "sm_mhz": mhz,
+            "peak_source": "measured: cp.async fills of random 512-B rows beside ldmatrix reads, "
+                           "84.1 B/clk/SM"}
 
 
-# L2 -> SM read peak of this B200, from the peak rates ncu reports for the kernel: 184 L2
-# slices (lts__cycles_elapsed.sum / .avg) x 2 sectors per slice clock
-# (lts__t_sectors_srcunit_tex peak_sustained) x 32 B x the 1.955 GHz L2 clock
-# (lts__cycles_elapsed.avg.per_second) = 23.0 TB/s
-L2_READ_PEAK_TBS = 184 * 2 * 32 * 1.955e9 / 1e12
-
-
-def _l2_bound(alg_bytes: int, t_s: float) -> dict:
-    """L2 read roofline: every algorithmic byte (gathered K/V rows, Q, indices) is read
-    from L2 by the SMs, hit or miss, against the ncu-derived L2 -> SM read peak."""
-    achieved = alg_bytes / t_s / 1e12
-    return {"bytes_per_launch": alg_bytes, "achieved": achieved, "peak": L2_READ_PEAK_TBS,
-            "unit": "TB/s", "frac": achieved / L2_READ_PEAK_TBS,
-            "peak_source": "ncu-derived: 184 L2 slices x 2 sectors/clk x 32 B x 1.955 GHz"}
+def _l2_bound(gathered: int, t_s: float, clk: dict, sms: int = 148) -> dict:
+    """L2 -> shared-memory gather bound: the gathered rows against the rate at which
+    cp.async alone brings random 512-byte rows of an L2-resident buffer into shared
+    memory (sms x 115.8 B per SM clock)."""
+    mhz = clk.get("sm_mhz") or 1965.0
+    peak = sms * GATHER_FILL_ALONE_B_PER_CLK * mhz * 1e6 / 1e12
+    achieved = gathered / t_s / 1e12
+    return {"bytes_per_launch": gathered, "achieved": achieved, "peak": peak,
+            "unit": "TB/s", "frac": achieved / peak, "sm_mhz": mhz,
+            "peak_source": "measured: cp.async fills of random 512-B rows from L2 alone, "
+                           "115.8 B/clk/SM"}
 
 
 def _kernel_hash():

@@ -367,7 +367,9 @@ def sparse_prefill_from_host(q, k_cache, v_cache, slot_idx, width=None, scale=No
     chunks of `chunk_rows`: chunk c+1's Q and indices cross the bus while chunk c is
     computed and chunk c-1's output returns on a third stream.  With nsplit = 0 every
     chunk uses the split plan of the whole batch, so the result is bitwise that of
-    sparse_prefill on the whole batch whatever the chunking.
+    sparse_prefill on the whole batch when the chunks launch the same kernel shape (a
+    launch of fewer waves may take another shape, which changes only the order of the
+    sums).
     """
     device = torch.device(device if device is not None else "cuda")
     if device.type != "cuda":
@@ -380,8 +382,8 @@ def sparse_prefill_from_host(q, k_cache, v_cache, slot_idx, width=None, scale=No
         # 5.83; chunks shrinking towards the end were slower still)
         chunk_rows = max(-(-Tq // 8), 256)
     if nsplit == 0:
-        # every chunk uses the whole batch's split plan, so the result does not depend
-        # on the chunking: it is bitwise that of one device call on the whole batch
+        # every chunk uses the whole batch's split plan (the kernel shape of a launch
+        # may still differ with its size, which changes only the order of the sums)
         num_sms = torch.cuda.get_device_properties(device).multi_processor_count
         nsplit, _ = qsa_sparse_prefill_block_plan(Tq, Hq, k_cache.shape[1], D, slot_idx.shape[1],
                                                   block, num_sms, 0)

@@ -224,13 +224,19 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
   if (uint64_t(k_stride_s) * kv_elem > UINT32_MAX || uint64_t(v_stride_s) * kv_elem > UINT32_MAX)
     return fail(QSA_ERR_UNSUPPORTED, "slot stride of 4 GiB or more");
 
-  int32_t num_sms = 0;
-  if (nsplit == 0) {
+  // the multiprocessor count sizes the automatic split plan (and, below, the kernel shape)
+  auto query_sms = [](int32_t& sms) -> qsa_status_t {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(QSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    num_sms = device_sm_count(dev);
-    if (num_sms <= 0) return fail(QSA_ERR_CUDA, "cannot query the multiprocessor count");
+    sms = device_sm_count(dev);
+    if (sms <= 0) return fail(QSA_ERR_CUDA, "cannot query the multiprocessor count");
+    return QSA_OK;
+  };
+  int32_t num_sms = 0;
+  if (nsplit == 0) {
+    const qsa_status_t st = query_sms(num_sms);
+    if (st != QSA_OK) return st;
   }
   const Plan pl = make_plan(Tq, Hq, Hkv, W, block, num_sms, nsplit);
   if (int64_t(Tq) * Hkv * pl.nsplit > int64_t(INT32_MAX))
@@ -242,6 +248,10 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
     if (!aligned16(workspace)) return fail(QSA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   }
 
+  if (num_sms == 0) {  // every argument is valid: only now touch the device
+    const qsa_status_t st = query_sms(num_sms);
+    if (st != QSA_OK) return st;
+  }
   qsa::FwdParams p{};
   p.q = static_cast<const uint16_t*>(q);
   p.k_cache = k_cache;
@@ -280,6 +290,7 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
   p.kv_fp8 = kv_fp8 ? 1 : 0;
   p.v_scale = kv_fp8 ? v_scale : 1.0f;
   p.head_major = qsa::kernel_order_head_major(S, Hkv, int32_t(kv_elem));
+  p.num_sms = num_sms;
   p.ent_lo = int32_t(part.slot_lo / block);
   p.ent_hi = int32_t((part.slot_lo + S) / block);
   p.ent_total = int32_t(S_total / block);

@@ -40,6 +40,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <type_traits>
 
 #include "qsa_internal.h"
 #include "qsa_ptx.cuh"
@@ -54,7 +55,7 @@ constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent)
 
 
-template <int NTILE, int DSPLIT, int SL, int STAGES, bool KV8 = false>
+template <int NTILE, int DSPLIT, int SL, int STAGES, bool KV8 = false, bool SLOT16 = false>
 struct Cfg {
   // warps serving one slot lane: a D-split pair (each warp handles every head tile over
   // its half of D) or one warp per head tile
@@ -68,15 +69,16 @@ struct Cfg {
   static constexpr int kStageBytes = SL * kSubBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;    // [slot lane][stage][sub-tile]
   static constexpr int kQBytes = NTILE * 8 * kRowBytes;
-  static constexpr int kIdxBytes = kMaxSlotsPerSplit * 4;  // compacted slot numbers
+  // compacted row numbers: 16-bit when the cache of the call has at most 65,536 rows
+  static constexpr int kIdxBytes = kMaxSlotsPerSplit * (SLOT16 ? 2 : 4);
   static constexpr int kScanBytes = 32 * 4;
   // partial scores a D-split pair exchanges when it also splits Q K^T: [lane][warp][32][4]
   static constexpr int kXchgBytes = (DSPLIT > 1) ? SL * DSPLIT * kTPW * 32 * 16 : 0;
   static constexpr int kTileFloats = 8 * kMergeStride + 16;  // one head tile's merge record
   static constexpr int kMergeBytes = kWarps * kTPW * kTileFloats * 4;
-  // with two head tiles per warp the exchange buffer overlays the Q tile, which is dead
-  // once the Q fragments are in registers
-  static constexpr bool kXchgOverQ = kTPW > 1;
+  // the exchange buffer overlays the Q tile, which is dead once the Q fragments are in
+  // registers
+  static constexpr bool kXchgOverQ = DSPLIT > 1;
   static_assert(!kXchgOverQ || kXchgBytes <= kQBytes, "exchange buffer fits the Q tile");
   static constexpr size_t kSmem =
       size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes + (kXchgOverQ ? 0 : kXchgBytes);
@@ -100,12 +102,13 @@ struct Cfg {
 // of the D index inside a k-step (Q K^T) or an m-tile (P V) is permuted to match what
 // ldmatrix delivers for 8-bit data; a sum over D does not depend on that order, and the
 // epilogue maps the m-tile rows back.
-template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8>
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8, bool SLOT16>
 __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p) {
   static_assert(!QSPLIT || DSPLIT == 2, "splitting Q K^T needs a D-split pair");
   constexpr int kKS = QSPLIT ? 8 : 16;  // k-steps of Q K^T per warp
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16>;
+  using SlotT = std::conditional_t<SLOT16, uint16_t, uint32_t>;
   constexpr int kKvRow = C::kKvRow;
   constexpr int kMT = 16 / DSPLIT;  // m16 tiles of D per warp in the PV product
   constexpr int TPW = C::kTPW;      // n8 head tiles per warp
@@ -113,7 +116,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   uint8_t* ring = smem;
   uint8_t* sQ = smem + C::kRingBytes;
   // Compacted valid slot numbers of the split, padded to whole 16-slot sub-tiles.
-  uint32_t* sSlot = reinterpret_cast<uint32_t*>(sQ + C::kQBytes);
+  SlotT* sSlot = reinterpret_cast<SlotT*>(sQ + C::kQBytes);
   int32_t* sScan = reinterpret_cast<int32_t*>(sSlot + kMaxSlotsPerSplit);
   float4* sXchg = C::kXchgOverQ ? reinterpret_cast<float4*>(sQ)  // (QSPLIT only)
                                  : reinterpret_cast<float4*>(sScan + 32);
@@ -208,7 +211,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
       const int v = sRaw[i];
       if (local(v)) {
         const uint32_t row = (uint32_t(v) - ent_lo) * uint32_t(block);  // row of this cache
-        for (int e = 0; e < block; ++e) sSlot[pos++] = row + uint32_t(e);
+        for (int e = 0; e < block; ++e) sSlot[pos++] = SlotT(row + uint32_t(e));
       }
     }
   }
@@ -268,15 +271,24 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   auto load_stage = [&](int s, int buf) {
     const int base = s * C::kRows + wslot * 16;
     if (base >= n_valid) return;  // an empty sub-tile is neither loaded nor read
-    const uint4* slots = reinterpret_cast<const uint4*>(sSlot + base + row0);  // 16-byte aligned
+    // rows i .. i + 3 of this warp's part of the sub-tile (one 16- or 8-byte read)
+    auto slots4 = [&](int i, uint32_t (&sl)[4]) {
+      if constexpr (SLOT16) {
+        const uint2 s2 = reinterpret_cast<const uint2*>(sSlot + base + row0)[i / 4];
+        sl[0] = s2.x & 0xffffu; sl[1] = s2.x >> 16; sl[2] = s2.y & 0xffffu; sl[3] = s2.y >> 16;
+      } else {
+        const uint4 s4 = reinterpret_cast<const uint4*>(sSlot + base + row0)[i / 4];
+        sl[0] = s4.x; sl[1] = s4.y; sl[2] = s4.z; sl[3] = s4.w;
+      }
+    };
     if constexpr (!KV8) {
       uint32_t kd[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m) kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (m << 4));
 #pragma unroll
       for (int i = 0; i < kLoadRows; i += 4) {
-        const uint4 s4 = slots[i / 4];  // slots of rows i .. i + 3
-        const uint32_t sl[4] = {s4.x, s4.y, s4.z, s4.w};
+        uint32_t sl[4];
+        slots4(i, sl);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t d = kd[(i + e) & 7] + (i + e) * kRowBytes;
@@ -292,9 +304,10 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
         kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (uint32_t((2 * m + lhalf) & 7) << 4));
 #pragma unroll
       for (int i = 0; i < kLoadRows; i += 4) {
-        const uint4 s4 = slots[i / 4];  // slots of rows i .. i + 3
-        const uint32_t sa = lhalf ? s4.y : s4.x;  // row i + lhalf
-        const uint32_t sb = lhalf ? s4.w : s4.z;  // row i + 2 + lhalf
+        uint32_t sl[4];
+        slots4(i, sl);
+        const uint32_t sa = lhalf ? sl[1] : sl[0];  // row i + lhalf
+        const uint32_t sb = lhalf ? sl[3] : sl[2];  // row i + 2 + lhalf
         const int ip = i / 2;
         uint32_t d = kd[ip & 3] + ip * 2 * kKvRow;
         cp_async_16_global(d, kg + uint64_t(sa) * kstride);
@@ -739,10 +752,11 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
   *reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8) = v;
 }
 
-template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8>
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8,
+          bool SLOT16 = false>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8>;
-  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16>;
+  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16>;
   // The shared-memory opt-in is a per-device function attribute: set it on the first
   // launch on each device only, so later calls (e.g. under stream capture) are launches
   // and nothing else.
@@ -818,6 +832,31 @@ static_assert(CfgLarge::kSmem <= CfgLarge::kSmPerCta(QSA_LARGE_CTAS), "large sha
 static_assert(CfgSmall8::kSmem <= CfgSmall8::kSmPerCta(QSA_SMALL_CTAS), "E4M3 small shape: CTAs per SM");
 static_assert(CfgLarge8::kSmem <= CfgLarge8::kSmPerCta(QSA_LARGE_CTAS), "E4M3 large shape: CTAs per SM");
 
+// Caches of at most 65,536 rows (the long prefill's among them): the compacted row list is
+// 16-bit, which brings a CTA of two slot lanes of two stages to 73 KB, so three such CTAs
+// (12 warps, as before) fit on an SM and hide one another's per-unit prologue and epilogue
+// better than two CTAs of three lanes (measured: long prefill 2.016 vs 2.096 ms, 512-slot
+// rows 0.317 vs 0.356 ms).  A CTA of two lanes takes ~1.4x as long per unit, so with few
+// units the coarser waves lose (4,000 units: 0.557 vs 0.564 ms; 2,048: 0.303 vs 0.297;
+// 512: 140 vs 102 us): the shape is used from eight of its waves on.  E4M3 caches keep
+// their shape with the 16-bit list.
+constexpr int64_t kRows16 = 65536;
+constexpr int64_t kShape16MinWaves = 8;
+#ifndef QSA_SMALL16_SL
+#define QSA_SMALL16_SL 2
+#endif
+#ifndef QSA_SMALL16_STAGES
+#define QSA_SMALL16_STAGES 2
+#endif
+#ifndef QSA_SMALL16_CTAS
+#define QSA_SMALL16_CTAS 3
+#endif
+using CfgSmall16 = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES, false, true>;
+using CfgSmall8r16 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true, true>;
+static_assert(CfgSmall16::kSmem <= CfgSmall16::kSmPerCta(QSA_SMALL16_CTAS), "16-bit shape: CTAs per SM");
+static_assert(CfgSmall8r16::kSmem <= CfgSmall8r16::kSmPerCta(QSA_SMALL_CTAS),
+              "E4M3 16-bit shape: CTAs per SM");
+
 }  // namespace
 
 KernelShape kernel_shape(int G) {
@@ -841,16 +880,29 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
 
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   cudaError_t e;
+  // every compacted row number is below the row count of this call's cache
+  const bool rows16 = p.S <= kRows16;
   if (p.kv_fp8) {
-    e = (p.G <= 8) ? launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
-                                true>(p, stream)
-                   : launch_fwd<2, QSA_LARGE_DSPLIT, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES,
-                                QSA_LARGE_CTAS, kLargeQsplit, true>(p, stream);
+    if (p.G <= 8)
+      e = rows16 ? launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
+                              true, true>(p, stream)
+                 : launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
+                              true>(p, stream);
+    else
+      e = launch_fwd<2, QSA_LARGE_DSPLIT, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, QSA_LARGE_CTAS,
+                     kLargeQsplit, true>(p, stream);
   } else {
-    e = (p.G <= 8) ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
-                                QSA_SMALL_QSPLIT, false>(p, stream)
-                   : launch_fwd<2, QSA_LARGE_DSPLIT, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS,
-                                kLargeQsplit, false>(p, stream);
+    const int64_t grid = int64_t(p.Tq) * p.Hkv * p.nsplit;
+    const bool shape16 =
+        rows16 && p.num_sms > 0 && grid >= kShape16MinWaves * p.num_sms * QSA_SMALL16_CTAS;
+    if (p.G <= 8)
+      e = shape16 ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES,
+                               QSA_SMALL16_CTAS, QSA_SMALL_QSPLIT, false, true>(p, stream)
+                  : launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
+                               QSA_SMALL_QSPLIT, false>(p, stream);
+    else
+      e = launch_fwd<2, QSA_LARGE_DSPLIT, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS,
+                     kLargeQsplit, false>(p, stream);
   }
   if (e != cudaSuccess || p.nsplit == 1) return e;
   return launch_combine(p, stream);

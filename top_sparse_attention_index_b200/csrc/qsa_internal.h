@@ -45,6 +45,7 @@ struct FwdParams {
   int32_t kv_fp8;           // 1: k_cache / v_cache hold E4M3 codes
   float v_scale;            // E4M3 cache: multiplier of the normalised output
   int32_t head_major;       // 1: work units ordered KV head slowest (see kernel_order)
+  int32_t num_sms;          // multiprocessors of the device (chooses the kernel shape)
   // Selected entries (slot numbers, or block numbers with block selection): an entry v is
   // valid when 0 <= v < ent_total and local when ent_lo <= v < ent_hi; the cache holds the
   // rows of the local entries, row (v - ent_lo) * block + e.  Unsharded: ent_lo = 0,

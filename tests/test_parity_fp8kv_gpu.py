@@ -321,3 +321,18 @@ def test_cache_offsets_beyond_4gib(cuda_device, oracle_lib):
     ref = oracle_lib.forward_fp8kv(q, rows_k, rows_v, idx_c, None, 1.0 / 16.0, KS, VS)
     check_gates(out.cpu().float(), torch.from_numpy(ref), None, "E4M3 cache past 4 GiB")
     del k_dev, v_dev
+
+
+@pytest.mark.parametrize("Hq,Hkv,S,nsplit", [(8, 2, 8192, 1), (6, 1, 30000, 3)])
+def test_many_wave_launches_with_masks_and_splits(cuda_device, oracle_lib, Hq, Hkv, S, nsplit):
+    """E4M3 launches of many waves (at least eight waves of three CTAs per SM) on caches of
+    at most 65,536 rows: ragged widths, interior -1 entries, an empty row, one split and
+    forced splits; the oracle's fp8 path checks every 7th row plus the first and last."""
+    Tq = 2400 if Hkv == 2 else 4000
+    w = _random_case(470 + Hq, Tq, Hq, Hkv, S, 300, minus1=0.1, widths=True)
+    w.slot_idx[5] = -1
+    d = dev(w, cuda_device)
+    got = run(w, d, 1.0 / 16.0, nsplit=nsplit)
+    rows = sorted(set(range(0, Tq, 7)) | {1, 5, Tq - 1})
+    compare(w, got, oracle_lib, 1.0 / 16.0, rows, f"E4M3 many waves Hq={Hq} S={S} nsplit={nsplit}")
+    assert torch.all(got[5] == 0)

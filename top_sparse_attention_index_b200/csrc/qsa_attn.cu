@@ -838,8 +838,9 @@ static_assert(CfgLarge8::kSmem <= CfgLarge8::kSmPerCta(QSA_LARGE_CTAS), "E4M3 la
 // better than two CTAs of three lanes (measured: long prefill 2.016 vs 2.096 ms, 512-slot
 // rows 0.317 vs 0.356 ms).  A CTA of two lanes takes ~1.4x as long per unit, so with few
 // units the coarser waves lose (4,000 units: 0.557 vs 0.564 ms; 2,048: 0.303 vs 0.297;
-// 512: 140 vs 102 us): the shape is used from eight of its waves on.  E4M3 caches keep
-// their shape with the 16-bit list.
+// 512: 140 vs 102 us): the shape is used from eight of its waves on.  E4M3 caches do the
+// same with two slot lanes of four stages (long prefill 1.756 vs 1.789 ms; with fewer waves
+// they keep four lanes of three stages, with the 16-bit list).
 constexpr int64_t kRows16 = 65536;
 constexpr int64_t kShape16MinWaves = 8;
 #ifndef QSA_SMALL16_SL
@@ -851,9 +852,18 @@ constexpr int64_t kShape16MinWaves = 8;
 #ifndef QSA_SMALL16_CTAS
 #define QSA_SMALL16_CTAS 3
 #endif
+#ifndef QSA_FP8_SMALL16_SL
+#define QSA_FP8_SMALL16_SL 2
+#endif
+#ifndef QSA_FP8_SMALL16_STAGES
+#define QSA_FP8_SMALL16_STAGES 4
+#endif
 using CfgSmall16 = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES, false, true>;
 using CfgSmall8r16 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true, true>;
+using CfgSmall8s16 = Cfg<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES, true, true>;
 static_assert(CfgSmall16::kSmem <= CfgSmall16::kSmPerCta(QSA_SMALL16_CTAS), "16-bit shape: CTAs per SM");
+static_assert(CfgSmall8s16::kSmem <= CfgSmall8s16::kSmPerCta(QSA_SMALL16_CTAS),
+              "E4M3 three-CTA shape: CTAs per SM");
 static_assert(CfgSmall8r16::kSmem <= CfgSmall8r16::kSmPerCta(QSA_SMALL_CTAS),
               "E4M3 16-bit shape: CTAs per SM");
 
@@ -882,19 +892,21 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   cudaError_t e;
   // every compacted row number is below the row count of this call's cache
   const bool rows16 = p.S <= kRows16;
+  const int64_t grid = int64_t(p.Tq) * p.Hkv * p.nsplit;
+  const bool shape16 =
+      rows16 && p.num_sms > 0 && grid >= kShape16MinWaves * p.num_sms * QSA_SMALL16_CTAS;
   if (p.kv_fp8) {
     if (p.G <= 8)
-      e = rows16 ? launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
-                              true, true>(p, stream)
-                 : launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
-                              true>(p, stream);
+      e = shape16 ? launch_fwd<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES, QSA_SMALL16_CTAS,
+                               true, true, true>(p, stream)
+          : rows16 ? launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
+                                true, true>(p, stream)
+                   : launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
+                                true>(p, stream);
     else
       e = launch_fwd<2, QSA_LARGE_DSPLIT, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, QSA_LARGE_CTAS,
                      kLargeQsplit, true>(p, stream);
   } else {
-    const int64_t grid = int64_t(p.Tq) * p.Hkv * p.nsplit;
-    const bool shape16 =
-        rows16 && p.num_sms > 0 && grid >= kShape16MinWaves * p.num_sms * QSA_SMALL16_CTAS;
     if (p.G <= 8)
       e = shape16 ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES,
                                QSA_SMALL16_CTAS, QSA_SMALL_QSPLIT, false, true>(p, stream)

@@ -55,7 +55,8 @@ constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent)
 
 
-template <int NTILE, int DSPLIT, int SL, int STAGES, bool KV8 = false, bool SLOT16 = false>
+template <int NTILE, int DSPLIT, int SL, int STAGES, bool KV8 = false, bool SLOT16 = false,
+          int QROWS = NTILE * 8>
 struct Cfg {
   // warps serving one slot lane: a D-split pair (each warp handles every head tile over
   // its half of D) or one warp per head tile
@@ -68,7 +69,11 @@ struct Cfg {
   static constexpr int kSubBytes = 16 * kKvRow * 2;          // one sub-tile: 16 K rows, 16 V rows
   static constexpr int kStageBytes = SL * kSubBytes;
   static constexpr int kRingBytes = STAGES * kStageBytes;    // [slot lane][stage][sub-tile]
-  static constexpr int kQBytes = NTILE * 8 * kRowBytes;
+  // the group's Q rows in shared memory: NTILE * 8, or fewer for a shape serving G <= QROWS
+  static constexpr int kQRows = QROWS;
+  static_assert(QROWS > (NTILE - 1) * 8 && QROWS <= NTILE * 8 && (!KV8 || QROWS == NTILE * 8),
+                "Q tile rows");
+  static constexpr int kQBytes = QROWS * kRowBytes;
   // compacted row numbers: 16-bit when the cache of the call has at most 65,536 rows
   static constexpr int kIdxBytes = kMaxSlotsPerSplit * (SLOT16 ? 2 : 4);
   static constexpr int kScanBytes = 32 * 4;
@@ -102,12 +107,13 @@ struct Cfg {
 // of the D index inside a k-step (Q K^T) or an m-tile (P V) is permuted to match what
 // ldmatrix delivers for 8-bit data; a sum over D does not depend on that order, and the
 // epilogue maps the m-tile rows back.
-template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8, bool SLOT16>
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8, bool SLOT16,
+          int QROWS>
 __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p) {
   static_assert(!QSPLIT || DSPLIT == 2, "splitting Q K^T needs a D-split pair");
   constexpr int kKS = QSPLIT ? 8 : 16;  // k-steps of Q K^T per warp
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16, QROWS>;
   using SlotT = std::conditional_t<SLOT16, uint16_t, uint32_t>;
   constexpr int kKvRow = C::kKvRow;
   constexpr int kMT = 16 / DSPLIT;  // m16 tiles of D per warp in the PV product
@@ -154,7 +160,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   const int64_t head0 = int64_t(j) * G;
   const uint32_t ring_s = smem_addr(ring);
   const uint32_t q_s = smem_addr(sQ);
-  for (int i = tid; i < NTILE * 8 * kChunks; i += C::kThreads) {
+  for (int i = tid; i < C::kQRows * kChunks; i += C::kThreads) {
     const int g = i / kChunks, c = i % kChunks;
     const bool ok = g < G;
     const uint16_t* src =
@@ -348,7 +354,14 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
         const int g = lane & 7;
         const int c = 4 * kp + 2 * ks0 + (lane >> 3);
         uint32_t r[4];
-        ldmatrix_x4(r, q_s + ((wn + nt) * 8 + g) * kRowBytes + ((c ^ g) << 4));
+        if constexpr (C::kQRows < NTILE * 8) {
+          // heads past the tile (>= QROWS >= G) are padding: their fragments are zero, and
+          // their row addresses stay inside the tile
+          ldmatrix_x4(r, q_s + min((wn + nt) * 8 + g, C::kQRows - 1) * kRowBytes + ((c ^ g) << 4));
+          if ((wn + nt) * 8 + (lane >> 2) >= C::kQRows) r[0] = r[1] = r[2] = r[3] = 0u;
+        } else {
+          ldmatrix_x4(r, q_s + ((wn + nt) * 8 + g) * kRowBytes + ((c ^ g) << 4));
+        }
         qf[nt][2 * kp][0] = r[0];
         qf[nt][2 * kp][1] = r[1];
         qf[nt][2 * kp + 1][0] = r[2];
@@ -753,10 +766,12 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
 }
 
 template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8,
-          bool SLOT16 = false>
+          bool SLOT16 = false, int QROWS = NTILE * 8>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16>;
-  auto kern = qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16, QROWS>;
+  if (p.G > QROWS) return cudaErrorInvalidValue;  // the Q tile holds the whole group
+  auto kern =
+      qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16, QROWS>;
   // The shared-memory opt-in is a per-device function attribute: set it on the first
   // launch on each device only, so later calls (e.g. under stream capture) are launches
   // and nothing else.
@@ -864,6 +879,15 @@ using CfgSmall8s16 = Cfg<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES, true,
 static_assert(CfgSmall16::kSmem <= CfgSmall16::kSmPerCta(QSA_SMALL16_CTAS), "16-bit shape: CTAs per SM");
 static_assert(CfgSmall8s16::kSmem <= CfgSmall8s16::kSmPerCta(QSA_SMALL16_CTAS),
               "E4M3 three-CTA shape: CTAs per SM");
+// 8 < G <= 12 on such caches: two slot lanes of two stages with a 12-row Q tile, three CTAs
+// per SM (G = 12: 2.518 vs 2.609 ms for 8,000 query rows of a 12,288-slot cache, 1.289 vs
+// 1.334 ms for 4,000 rows of 65,536 slots; G = 10 2.515 vs 2.604 ms).
+#ifndef QSA_LARGE16_QROWS
+#define QSA_LARGE16_QROWS 12
+#endif
+using CfgLarge16 = Cfg<2, 2, 2, 2, false, true, QSA_LARGE16_QROWS>;
+static_assert(CfgLarge16::kSmem <= CfgLarge16::kSmPerCta(QSA_SMALL16_CTAS),
+              "12-row two-tile shape: CTAs per SM");
 static_assert(CfgSmall8r16::kSmem <= CfgSmall8r16::kSmPerCta(QSA_SMALL_CTAS),
               "E4M3 16-bit shape: CTAs per SM");
 
@@ -912,6 +936,8 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
                                QSA_SMALL16_CTAS, QSA_SMALL_QSPLIT, false, true>(p, stream)
                   : launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
                                QSA_SMALL_QSPLIT, false>(p, stream);
+    else if (shape16 && p.G <= QSA_LARGE16_QROWS)
+      e = launch_fwd<2, 2, 2, 2, QSA_SMALL16_CTAS, true, false, true, QSA_LARGE16_QROWS>(p, stream);
     else
       e = launch_fwd<2, QSA_LARGE_DSPLIT, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS,
                      kLargeQsplit, false>(p, stream);

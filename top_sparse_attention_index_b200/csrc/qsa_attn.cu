@@ -487,9 +487,10 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     // With one head tile per warp the first kVEarly V fragments of the sub-tile (bf16: m-tiles;
     // E4M3: raw codes of m-tile pairs) are read here, before the score exchange and the
     // softmax, so their shared-memory latency is hidden behind that work (the stage has
-    // landed; the registers fit under the two-CTA cap).  With two head tiles per warp the
-    // registers are already at the cap and the early reads cost more than they hide.
-    constexpr int kVEarly = TPW == 1 ? (KV8 ? 2 : 4) : 0;
+    // landed; the registers fit under the cap).  The E4M3 shape of two slot lanes has the
+    // registers for all of its pairs (measured 1.738 vs 1.759 ms).  With two head tiles per
+    // warp the registers are already at the cap and the early reads cost more than they hide.
+    constexpr int kVEarly = TPW == 1 ? (KV8 ? (SL == 2 ? kMT / 2 : 2) : 4) : 0;
     uint32_t vt[4];
     uint32_t vearly[kVEarly > 0 ? kVEarly : 1][4];
 #pragma unroll

@@ -471,13 +471,23 @@ def _l2_bound(gathered: int, t_s: float, clk: dict, sms: int = 148) -> dict:
                            "115.8 B/clk/SM"}
 
 
+def _code_only(text: str) -> str:
+    """C++ source with comments removed and whitespace collapsed (string and character
+    literals kept), so that editing a comment does not change the kernel's hash."""
+    import re
+    token = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"|\'(?:\\.|[^\'\\])*\'', re.S)
+    text = token.sub(lambda m: " " if m.group(0).startswith("/") else m.group(0), text)
+    return " ".join(text.split())
+
+
 def _kernel_hash():
-    """Hash of the kernel sources (the DRAM traffic record is valid while it matches)."""
+    """Hash of the kernel code, comments and whitespace aside (the DRAM traffic record
+    is valid while it matches)."""
     import hashlib
     h = hashlib.sha256()
     csrc = ROOT / "top_sparse_attention_index_b200" / "csrc"
     for name in ("qsa_attn.cu", "qsa_internal.h", "qsa_ptx.cuh"):
-        h.update((csrc / name).read_bytes())
+        h.update(_code_only((csrc / name).read_text()).encode())
     return h.hexdigest()[:16]
 
 

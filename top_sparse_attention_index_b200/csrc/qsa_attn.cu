@@ -6,10 +6,11 @@
 // scale * Q K^T for the whole GQA group of G = Hq / Hkv query heads, take the softmax
 // over the selected slots only and return P V; a row without a valid slot returns 0.
 //
-// K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit, two CTAs
-// resident per SM so that one CTA's prologue and epilogue overlap the other's gather
-// (units ordered KV head slowest when one head's slice of the cache fits L2 and the
-// whole cache does not):
+// K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit, two or three CTAs
+// resident per SM so that one CTA's prologue and epilogue overlap the others' gathers
+// (three, of two slot lanes each, when the cache has at most 65,536 rows so the compacted
+// row list is 16-bit, and the launch has many waves; units ordered KV head slowest when
+// one head's slice of the cache fits L2 and the whole cache does not):
 //   1. stage the split's slot indices in shared memory and compact away -1 (and
 //      out-of-range) entries with a block scan, so masked slots cost no bandwidth;
 //   2. gather K and V rows of the compacted slots with 16-byte cp.async into shared

@@ -884,10 +884,16 @@ static_assert(CfgSmall8s16::kSmem <= CfgSmall8s16::kSmPerCta(QSA_SMALL16_CTAS),
 // 8 < G <= 12 on such caches: two slot lanes of two stages with a 12-row Q tile, three CTAs
 // per SM (G = 12: 2.518 vs 2.609 ms for 8,000 query rows of a 12,288-slot cache, 1.289 vs
 // 1.334 ms for 4,000 rows of 65,536 slots; G = 10 2.515 vs 2.604 ms).
+#ifndef QSA_LARGE16_SL
+#define QSA_LARGE16_SL 2
+#endif
+#ifndef QSA_LARGE16_STAGES
+#define QSA_LARGE16_STAGES 2
+#endif
 #ifndef QSA_LARGE16_QROWS
 #define QSA_LARGE16_QROWS 12
 #endif
-using CfgLarge16 = Cfg<2, 2, 2, 2, false, true, QSA_LARGE16_QROWS>;
+using CfgLarge16 = Cfg<2, 2, QSA_LARGE16_SL, QSA_LARGE16_STAGES, false, true, QSA_LARGE16_QROWS>;
 static_assert(CfgLarge16::kSmem <= CfgLarge16::kSmPerCta(QSA_SMALL16_CTAS),
               "12-row two-tile shape: CTAs per SM");
 static_assert(CfgSmall8r16::kSmem <= CfgSmall8r16::kSmPerCta(QSA_SMALL_CTAS),
@@ -914,6 +920,9 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
   return workspace_lse_offset(Tq, Hq, nsplit) + (lse_bytes + 255) / 256 * 256;
 }
 
+// Kernel shape of a call: by cache format and group size G; caches of at most 65,536 rows
+// take the 16-bit row list, and with it, in launches of at least eight waves, the shapes of
+// three CTAs per SM (G <= 8, and 8 < G <= 12 for bf16 caches).
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   cudaError_t e;
   // every compacted row number is below the row count of this call's cache
@@ -939,7 +948,8 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
                   : launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
                                QSA_SMALL_QSPLIT, false>(p, stream);
     else if (shape16 && p.G <= QSA_LARGE16_QROWS)
-      e = launch_fwd<2, 2, 2, 2, QSA_SMALL16_CTAS, true, false, true, QSA_LARGE16_QROWS>(p, stream);
+      e = launch_fwd<2, 2, QSA_LARGE16_SL, QSA_LARGE16_STAGES, QSA_SMALL16_CTAS, true, false, true,
+                     QSA_LARGE16_QROWS>(p, stream);
     else
       e = launch_fwd<2, QSA_LARGE_DSPLIT, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS,
                      kLargeQsplit, false>(p, stream);

@@ -76,3 +76,32 @@ def test_reference_arm_runs_on_rank0_only(capsys):
         gpus, steps, warmup = 2, 1, 0
     assert bench.run_reference(A(), rank=1) is None
     assert capsys.readouterr().out == ""
+
+
+def test_kernel_hash_ignores_comments_and_whitespace():
+    """The traffic record's key: comments and layout do not change it, code does, and
+    string or character literals that look like comments are kept."""
+    a = 'int f() { return 1; } // one\n/* block\n comment */ const char* s = "// x";'
+    b = 'int  f()  {\n  return 1;  }\nconst char* s = "// x"; // other comment'
+    c = 'int f() { return 2; } const char* s = "// x";'
+    d = 'int f() { return 1; } const char* s = "// y";'
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert bench._code_only(a) != bench._code_only(d)
+    assert bench._code_only("char q = '/'; // c") == "char q = '/';"
+    assert len(bench._kernel_hash()) == 16
+
+
+def test_sm_side_bounds_scale_with_the_sampled_clock():
+    """The shared-memory and L2 bounds are the measured per-SM byte rates times 148 SMs
+    times the sampled clock; the fractions are achieved / peak."""
+    gathered, t = 32.8e9, 2.0e-3
+    for fn, rate in ((bench._smem_bound, bench.GATHER_FILL_WITH_READS_B_PER_CLK),
+                     (bench._l2_bound, bench.GATHER_FILL_ALONE_B_PER_CLK)):
+        r = fn(gathered, t, {"sm_mhz": 1965.0})
+        assert abs(r["peak"] - 148 * rate * 1.965e9 / 1e12) < 1e-9
+        assert abs(r["achieved"] - gathered / t / 1e12) < 1e-9
+        assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
+        slow = fn(gathered, t, {"sm_mhz": 1000.0})
+        assert abs(slow["peak"] / r["peak"] - 1000.0 / 1965.0) < 1e-12
+        assert fn(gathered, t, {"sm_mhz": None})["sm_mhz"] == 1965.0  # unsampled: max clock

@@ -718,13 +718,21 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
 }
 
 // K2: out[t, h, :] = sum_s 2^(lse_s - lse*) O_s / sum_s 2^(lse_s - lse*), one warp per row.
+// The lanes read the splits' LSEs side by side (lane i: splits i, i + 32, ...) and reduce
+// their maximum; the weighted sum then runs over the splits in order, every lane adding
+// its eight elements of D, with the partial rows read regardless of their weight (the
+// buffers hold every split's row) so that the reads of several splits are in flight at
+// once; a split with lse = -inf (empty, its row never written) is left out by a select.
 __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p) {
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   const int64_t row = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int lane = threadIdx.x & 31;
+  const int ns = p.nsplit;
   float mstar = kNegInf;
-  for (int s = 0; s < p.nsplit; ++s) mstar = fmaxf(mstar, p.ws_lse[s * rows + row]);
+  for (int s = lane; s < ns; s += 32) mstar = fmaxf(mstar, p.ws_lse[s * rows + row]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, off));
   const int64_t t = row / p.Hq, h = row % p.Hq;
   if (mstar == kNegInf) {  // no valid slot in any split
     if (p.partial_out) {
@@ -741,15 +749,22 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   float wsum = 0.f;
-  for (int s = 0; s < p.nsplit; ++s) {
-    const float lse = p.ws_lse[s * rows + row];
-    if (lse == kNegInf) continue;  // empty split: its partial was never written
-    const float w = fast_exp2(lse - mstar);
-    wsum += w;
-    const float4* src = reinterpret_cast<const float4*>(p.ws_o + (s * rows + row) * kHeadDim + lane * 8);
-    const float4 a = src[0], b = src[1];
-    acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
-    acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    const float lse_l = s0 + lane < ns ? p.ws_lse[(s0 + lane) * rows + row] : kNegInf;
+    const int cnt = min(32, ns - s0);
+#pragma unroll 4
+    for (int i = 0; i < cnt; ++i) {
+      const float lse = __shfl_sync(0xffffffffu, lse_l, i);
+      const float4* src =
+          reinterpret_cast<const float4*>(p.ws_o + ((s0 + i) * rows + row) * kHeadDim + lane * 8);
+      const float4 a = src[0], b = src[1];
+      if (lse != kNegInf) {  // warp-uniform
+        const float w = fast_exp2(lse - mstar);
+        wsum += w;
+        acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+        acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
+      }
+    }
   }
   const float inv = 1.f / wsum;
   if (p.partial_out) {  // one normalised record of all splits: O and lse* + log2(sum of weights)

@@ -93,6 +93,18 @@ int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, 
                                 size_t* workspace_bytes);
 
 /*
+ * qsa_sparse_prefill_workspace_bytes -- workspace size of the automatic plan.
+ *
+ * Host only, like qsa_sparse_prefill_plan, of which it is the nsplit_request == 0 case
+ * with the arguments in the order (Tq, Hq, Hkv, W, D, num_sms): the bytes of device
+ * scratch that qsa_sparse_prefill with nsplit == 0 needs on a device of `num_sms`
+ * multiprocessors (0 when the plan does not split W).  Returns SIZE_MAX when the shape
+ * is invalid or unsupported (qsa_last_error_detail() says why).
+ */
+size_t qsa_sparse_prefill_workspace_bytes(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W,
+                                          int32_t D, int32_t num_sms);
+
+/*
  * qsa_sparse_prefill -- selected-slot sparse attention for one prefill batch.
  *
  * Arguments (all device pointers unless stated):
@@ -276,16 +288,20 @@ qsa_status_t qsa_combine_partials(const float* part_o, const float* part_lse, in
  * Arguments, layouts, ownership and errors are those of qsa_sparse_prefill without
  * `workspace` / `workspace_bytes`.  It calls no cudaMalloc, cudaFree or other
  * allocating routine.  Additional behaviour:
- *   - the first call on a device (the current device) looks up that device's address
- *     of the scratch array (cudaGetSymbolAddress) and caches it; make that first call
- *     before any stream capture on the device;
+ *   - the first call on a device (the current device) that needs scratch looks up that
+ *     device's address of the array (cudaGetSymbolAddress) and caches it under the
+ *     current CUDA context's unique ID; make that first call before any stream capture
+ *     on the device.  After a device reset (or with another context current) the
+ *     address is looked up again on the next call, so no stale address is used;
  *   - a shape whose plan needs more scratch than QSA_STATIC_SCRATCH_BYTES returns
  *     QSA_ERR_WORKSPACE before any launch (qsa_sparse_prefill_plan gives the need;
  *     a smaller nsplit request, or the workspace entry point, are the ways out);
  *   - all calls on a device share the one array and it keeps whatever the last call
- *     left in it; nothing in it has to start at zero (every value a call reads was
- *     written earlier in the same call), but calls whose kernels overlap on the GPU
- *     (e.g. on two streams) race on it: serialise them.
+ *     left in it; nothing in it has to start at zero: every log-sum-exp value a call
+ *     reads was written earlier in the same call, and a split's partial output row is
+ *     read but ignored when that split's log-sum-exp is -inf (an empty split, whose row
+ *     the call does not write), so stale contents never reach `out`.  Calls whose
+ *     kernels overlap on the GPU (e.g. on two streams) race on the array: serialise them.
  */
 qsa_status_t qsa_sparse_prefill_noalloc(const void* q, int64_t q_stride_t, int64_t q_stride_h,
                                         const void* k_cache, int64_t k_stride_s,

@@ -101,6 +101,32 @@ def test_plan_wide_rows_force_splits(lib):
     assert n == 1 and ws == 0
 
 
+@pytest.mark.parametrize("Tq,Hq,Hkv,W", [
+    (7810, 16, 2, 2051), (16, 16, 2, 2051), (1, 16, 2, 2051), (257, 12, 1, 2051),
+    (100000, 16, 2, 6000), (10, 16, 2, 0), (64, 6, 1, 2048),
+])
+def test_workspace_bytes_is_the_automatic_plan(lib, Tq, Hq, Hkv, W):
+    # the raw C call, argument order (Tq, Hq, Hkv, W, D, num_sms)
+    raw = lib.qsa_sparse_prefill_workspace_bytes(Tq, Hq, Hkv, W, 256, 148)
+    _, ws = qsa.qsa_sparse_prefill_plan(Tq, Hq, Hkv, 256, W, 148)
+    assert raw == ws
+    assert qsa.qsa_sparse_prefill_workspace_bytes(Tq, Hq, Hkv, W, 256, 148) == ws
+
+
+@pytest.mark.parametrize("shape,status", [
+    ((4, 16, 3, 8, 256), qsa.QSA_ERR_INVALID_ARG),   # Hq % Hkv
+    ((4, 16, 2, 8, 128), qsa.QSA_ERR_UNSUPPORTED),   # D != 256
+    ((4, 17, 1, 8, 256), qsa.QSA_ERR_UNSUPPORTED),   # G = 17
+    ((-1, 16, 2, 8, 256), qsa.QSA_ERR_INVALID_ARG),  # negative Tq
+])
+def test_workspace_bytes_rejects(lib, shape, status):
+    assert lib.qsa_sparse_prefill_workspace_bytes(*shape, 148) == ctypes.c_size_t(-1).value
+    assert qsa.qsa_last_error_detail() != ""
+    with pytest.raises(qsa.QSAError) as ei:
+        qsa.qsa_sparse_prefill_workspace_bytes(*shape, 148)
+    assert ei.value.status == status
+
+
 @pytest.mark.parametrize("shape,status", [
     ((4, 16, 3, 256, 8), qsa.QSA_ERR_INVALID_ARG),   # Hq % Hkv
     ((4, 16, 2, 128, 8), qsa.QSA_ERR_UNSUPPORTED),   # D != 256

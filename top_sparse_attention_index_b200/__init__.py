@@ -29,6 +29,7 @@ from ._binding import (  # noqa: F401
     qsa_sparse_prefill_partial,
     qsa_sparse_prefill_noalloc,
     qsa_sparse_prefill_plan,
+    qsa_sparse_prefill_workspace_bytes,
     qsa_status_string,
     combine_partials,
     sparse_prefill,
@@ -42,6 +43,6 @@ __all__ = [
     "qsa_sparse_prefill_block", "qsa_sparse_prefill_block_plan", "qsa_sparse_prefill_fp8kv",
     "qsa_sparse_prefill_partial", "qsa_combine_partials", "sparse_prefill_partial",
     "combine_partials", "sparse_prefill_context_parallel", "shard_ranges",
-    "qsa_sparse_prefill_plan", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
+    "qsa_sparse_prefill_plan", "qsa_sparse_prefill_workspace_bytes", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
     "load_library", "QSAError",
 ]

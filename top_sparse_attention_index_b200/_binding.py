@@ -31,6 +31,7 @@ _p, _i32, _i64, _sz, _f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctype
 SIGNATURES = {
     "qsa_abi_version": (_i32, []),
     "qsa_sparse_prefill_plan": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.POINTER(_sz)]),
+    "qsa_sparse_prefill_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "qsa_sparse_prefill": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p, _i64, _p,
                                   _i32, _i32, _i32, _i32, _i64, _i32, _f, _p, _i64, _i64, _i32,
                                   _p, _sz, _p, _p]),
@@ -105,6 +106,15 @@ def qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms, nsplit_request=0):
     if n < 0:
         raise QSAError(-n, qsa_last_error_detail())
     return n, int(ws.value)
+
+
+def qsa_sparse_prefill_workspace_bytes(Tq, Hq, Hkv, W, D, num_sms) -> int:
+    """Workspace bytes of the automatic plan; raises QSAError for invalid shapes."""
+    n = int(load_library().qsa_sparse_prefill_workspace_bytes(Tq, Hq, Hkv, W, D, num_sms))
+    if n == ctypes.c_size_t(-1).value:
+        qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms)  # raises with the status
+        raise QSAError(QSA_ERR_INVALID_ARG, qsa_last_error_detail())
+    return n
 
 
 def qsa_sparse_prefill(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,

@@ -5,6 +5,7 @@
 // the scalar arguments and pointer values, so a call is a pure enqueue on `stream`
 // (unlike the Ascend adapter described in "What the pull request actually adds",
 // whose extent check copies two scalars to the host).
+#include <cuda.h>  // driver types of the context-ID query (resolved at run time)
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -111,6 +112,39 @@ void set_error_detail(const char* fmt, ...) {
   std::vsnprintf(g_detail, sizeof g_detail, fmt, ap);
   va_end(ap);
 }
+
+// The two driver entry points are looked up through the runtime once per process, so the
+// library needs no link-time dependency on libcuda.
+uint64_t current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  struct Fns {
+    GetCurrentFn get_current = nullptr;
+    GetIdFn get_id = nullptr;
+  };
+  static const Fns fns = [] {
+    Fns f;
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult ra{}, rb{};
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &a, 12000, cudaEnableDefault, &ra) ==
+            cudaSuccess &&
+        ra == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPointByVersion("cuCtxGetId", &b, 12000, cudaEnableDefault, &rb) ==
+            cudaSuccess &&
+        rb == cudaDriverEntryPointSuccess) {
+      f.get_current = reinterpret_cast<GetCurrentFn>(a);
+      f.get_id = reinterpret_cast<GetIdFn>(b);
+    }
+    return f;
+  }();
+  if (fns.get_current == nullptr || fns.get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (fns.get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (fns.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(id);
+}
 }  // namespace qsa
 
 extern "C" {
@@ -147,6 +181,13 @@ int32_t qsa_sparse_prefill_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, 
                                 size_t* workspace_bytes) {
   return qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, 1, num_sms, nsplit_request,
                                        workspace_bytes);
+}
+
+size_t qsa_sparse_prefill_workspace_bytes(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t W,
+                                          int32_t D, int32_t num_sms) {
+  size_t bytes = 0;
+  if (qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms, 0, &bytes) < 0) return SIZE_MAX;
+  return bytes;
 }
 
 }  // extern "C"

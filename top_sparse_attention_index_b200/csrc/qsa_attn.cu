@@ -789,19 +789,24 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
   if (p.G > QROWS) return cudaErrorInvalidValue;  // the Q tile holds the whole group
   auto kern =
       qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16, QROWS>;
-  // The shared-memory opt-in is a per-device function attribute: set it on the first
-  // launch on each device only, so later calls (e.g. under stream capture) are launches
-  // and nothing else.
-  static std::atomic<uint64_t> configured{0};
+  // The shared-memory opt-in is a function attribute that lives in the CUDA context: set
+  // it on the first launch in each context only (keyed by the context's unique ID, so a
+  // device reset or a new context sets it again), so later calls (e.g. under stream
+  // capture) are launches and nothing else.
+  static std::atomic<uint64_t> configured_ctx[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
-  if (bit == 0 || !(configured.load(std::memory_order_acquire) & bit)) {
+  const uint64_t ctx = current_context_id();
+  const bool cached = dev >= 0 && dev < 64 && ctx != 0 &&
+                      configured_ctx[dev].load(std::memory_order_acquire) == ctx;
+  if (!cached) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(C::kSmem));
     if (e != cudaSuccess) return e;
-    configured.fetch_or(bit, std::memory_order_acq_rel);
+    // (the attribute call made the context current if no call had before)
+    const uint64_t now = current_context_id();
+    if (dev >= 0 && dev < 64 && now != 0) configured_ctx[dev].store(now, std::memory_order_release);
   }
   const unsigned grid = static_cast<unsigned>(int64_t(p.Tq) * p.Hkv * p.nsplit);
   kern<<<grid, C::kThreads, C::kSmem, stream>>>(p);

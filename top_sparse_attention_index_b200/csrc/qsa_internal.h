@@ -95,6 +95,13 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit);
 
 // printf-style detail for qsa_last_error_detail() on the calling host thread.
 void set_error_detail(const char* fmt, ...);
+
+// Process-unique identifier of the CUDA context current on the calling thread (the
+// driver's context ID), or 0 when none is current or the driver cannot say.  Per-device
+// state that lives in a context (a symbol's device address, a kernel's function
+// attributes) is cached under this ID, so a device reset or a new primary context
+// invalidates the cache instead of leaving stale addresses behind.
+uint64_t current_context_id();
 size_t workspace_lse_offset(int32_t Tq, int32_t Hq, int32_t nsplit);
 
 }  // namespace qsa

@@ -21,15 +21,23 @@ namespace {
 // The shared scratch: fp32 split partials and base-2 log-sum-exp values.  Host code
 // must never pass `g_static_scratch` itself to a kernel: on the host that name is only
 // a stand-in for the symbol, not a device address.  The address comes from
-// cudaGetSymbolAddress, once per device.
+// cudaGetSymbolAddress, once per device (and again after the device's context changes).
 static __device__ __align__(256) unsigned char g_static_scratch[QSA_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
+// Per device: the context the address was looked up in (its process-unique ID) and the
+// address.  A device reset or any new context on the device changes the ID, and the next
+// call looks the address up again instead of reusing one that is no longer mapped.
+struct ScratchSlot {
+  uint64_t ctx_id = 0;
+  void* addr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mutex;
 
-// Device address of the scratch array on the current device (looked up on the first
-// call per device, with that device current, then cached).
+// Device address of the scratch array in the context current on the calling thread:
+// looked up with cudaGetSymbolAddress on the first call per device (with that device
+// current) and again whenever the device's context has changed since; cached otherwise.
 qsa_status_t scratch_address(void** addr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -43,7 +51,9 @@ qsa_status_t scratch_address(void** addr) {
     return QSA_ERR_UNSUPPORTED;
   }
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchSlot& slot = g_scratch[dev];
+  const uint64_t ctx = qsa::current_context_id();
+  if (ctx == 0 || slot.addr == nullptr || slot.ctx_id != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess || p == nullptr) {
@@ -51,9 +61,11 @@ qsa_status_t scratch_address(void** addr) {
                             cudaGetErrorString(e));
       return QSA_ERR_CUDA;
     }
-    g_scratch_addr[dev] = p;
+    // (the lookup makes the device's context current if nothing had before)
+    slot.ctx_id = qsa::current_context_id();
+    slot.addr = p;
   }
-  *addr = g_scratch_addr[dev];
+  *addr = slot.addr;
   return QSA_OK;
 }
 

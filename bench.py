@@ -374,22 +374,25 @@ def main():
         e2e = {"value": world * flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # the SM-side roofline, measured right after the timed region on the same device
+    probe = gather_peak(device, 256 if w.kv_format == "e4m3" else 512)
+
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return
 
-    peak, peak_kind = measured_peaks()
+    hbm_peak, peak_kind = measured_peaks()
     t_s = ms_per_step * 1e-3
     achieved = alg_bytes / t_s / 1e9
-    traffic = None
+    traffic, ncu_rec = None, None
     prof = ROOT / "profiles" / "traffic.json"
     if prof.exists():
         # one record per workload; a record counts only while the kernel sources it was
         # captured with are unchanged
         for rec in json.loads(prof.read_text()).get("records", []):
             if rec.get("kernel_source_hash") == _kernel_hash() and rec.get("workload_name") == w.name:
-                traffic = rec.get("bytes_per_launch")
+                traffic, ncu_rec = rec.get("bytes_per_launch"), rec
     result = {
         "metric": METRIC,
         "value": world * flops / t_s / 1e12,
@@ -411,16 +414,22 @@ def main():
         "pairs_per_s": world * pairs / t_s,
         "pairs_x_hkv_per_s": world * pairs * w.Hkv / t_s,
         "gathered_gb_per_s": gathered / t_s / 1e9,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_source": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": alg_bytes},
-        # the bounds that bind once the gathered rows are L2 hits: the rate at which
-        # shared memory takes the copied rows while they are read back, and the L2 ->
-        # shared-memory gather rate alone
-        "shared_memory": _smem_bound(gathered, t_s, clocks.summary(t0_epoch, t1_epoch)),
-        # the bound of the L2-resident gather (most gathered rows are L2 hits)
-        "l2": _l2_bound(gathered, t_s, clocks.summary(t0_epoch, t1_epoch)),
+        # the bound that binds: the gather of L2-resident rows into shared memory (the
+        # cache is about the size of L2, so nearly every gathered row is an L2 hit);
+        # peak = the best rate of the gather probe, measured live on this device
+        "roofline": {"bound": "l2", "achieved": achieved, "peak": probe["tb_per_s"] * 1e3,
+                     "unit": "GB/s", "frac": achieved / (probe["tb_per_s"] * 1e3),
+                     "traffic": traffic, "algorithmic_bytes_per_launch": alg_bytes,
+                     "peak_source": "measured live: gather probe (qsa_probe_gather), best of "
+                                    f"{len(probe['runs'])} pipeline shapes: {probe['best']}",
+                     "ncu_l2_throughput_pct": (ncu_rec or {}).get(
+                         "lts__throughput.avg.pct_of_peak_sustained_elapsed")},
+        # HBM: the DRAM bytes the launch actually moves (ncu, one full-size launch of the
+        # current kernel code) against the measured copy bandwidth
+        "hbm": {"achieved": traffic / t_s / 1e9 if traffic else None, "peak": hbm_peak,
+                "unit": "GB/s", "frac": traffic / t_s / 1e9 / hbm_peak if traffic else None,
+                "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
+        "gather_probe": probe,
         "warm_l2": {"ms_per_step_median": warm_ms, "launches": n_warm,
                     "value": world * flops / (warm_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "note": "no L2 flush between launches; not the timed region"},
@@ -435,40 +444,62 @@ def main():
     print(json.dumps(result))
 
 
-# Shared-memory and L2 rates of this B200, measured by a probe with the gather's access
-# pattern (one CTA of 16 warps per SM; cp.async.cg copies of random 512-byte rows of an
-# L2-resident 64 MB buffer into shared memory, ldmatrix.x4 reads of shared memory; cycles
-# by clock64):  fills alone 115.8 B per SM clock, ldmatrix reads alone 126.3; both at once
-# 84.1 B/clk of fills beside 98.5 of reads.
-GATHER_FILL_ALONE_B_PER_CLK = 115.8
-GATHER_FILL_WITH_READS_B_PER_CLK = 84.1
+# The gather probe (include/qsa_probe.h) measures, live on the device, the rate at which
+# the SMs pull random rows of an L2-resident 64 MB buffer into shared memory and read each
+# landed row back once with ldmatrix -- the data movement of the fused kernel without its
+# arithmetic -- with the fused kernel's own loader (cp.async, method 0) and with TMA
+# tile::gather4 (method 1), over a few pipeline shapes (warps per CTA, stages, CTAs per
+# SM).  The best rate is the SM-side roofline of a launch whose gathered rows are L2 hits.
+PROBE_BUFFER_BYTES = 64 << 20
+PROBE_CONFIGS = {
+    512: [(12, 2, 1), (8, 3, 1), (6, 2, 2), (2, 4, 3)],
+    256: [(15, 3, 1), (12, 4, 1), (4, 4, 3), (6, 4, 2)],
+}
 
 
-def _smem_bound(gathered: int, t_s: float, clk: dict, sms: int = 148) -> dict:
-    """Shared-memory bound of the gather: every gathered byte is copied into shared memory
-    (cp.async) and read back once (ldmatrix); with both streams equal, the fill rate
-    measured beside concurrent reads binds (sms x 84.1 B per SM clock at the median SM
-    clock sampled during the timed region)."""
-    mhz = clk.get("sm_mhz") or 1965.0
-    peak = sms * GATHER_FILL_WITH_READS_B_PER_CLK * mhz * 1e6 / 1e12
-    achieved = gathered / t_s / 1e12
-    return {"bytes_per_launch": gathered, "achieved": achieved, "peak": peak,
-            "unit": "TB/s", "frac": achieved / peak, "sm_mhz": mhz,
-            "peak_source": "measured: cp.async fills of random 512-B rows beside ldmatrix reads, "
-                           "84.1 B/clk/SM"}
+def gather_peak(device, row_bytes: int, reps: int = 5) -> dict:
+    """Best gather rate (TB/s) of the probe over its methods and pipeline shapes."""
+    import top_sparse_attention_index_b200 as qsa
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    gen = torch.Generator(device=device).manual_seed(99)
+    buf = torch.randint(-2**31, 2**31 - 1, (PROBE_BUFFER_BYTES // 4,), dtype=torch.int32,
+                        device=device, generator=gen)
+    sink = torch.zeros(258, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    rows = PROBE_BUFFER_BYTES // row_bytes
+    runs = []
+    for method in (0, 1):
+        for warps, stages, per_sm in PROBE_CONFIGS[row_bytes]:
+            ctas = sms * per_sm
+            iters = max(4, int(2e9 / (ctas * warps * 16 * row_bytes)))
+            moved = ctas * warps * iters * 16 * row_bytes
+            sink.zero_()
 
+            def launch(seed):
+                st = qsa.qsa_probe_gather(method, 1, buf.data_ptr(), rows, row_bytes, row_bytes,
+                                          warps, stages, ctas, iters, seed, sink.data_ptr(),
+                                          stream.cuda_stream)
+                if st != qsa.QSA_OK:
+                    raise qsa.QSAError(st, qsa.qsa_last_error_detail())
 
-def _l2_bound(gathered: int, t_s: float, clk: dict, sms: int = 148) -> dict:
-    """L2 -> shared-memory gather bound: the gathered rows against the rate at which
-    cp.async alone brings random 512-byte rows of an L2-resident buffer into shared
-    memory (sms x 115.8 B per SM clock)."""
-    mhz = clk.get("sm_mhz") or 1965.0
-    peak = sms * GATHER_FILL_ALONE_B_PER_CLK * mhz * 1e6 / 1e12
-    achieved = gathered / t_s / 1e12
-    return {"bytes_per_launch": gathered, "achieved": achieved, "peak": peak,
-            "unit": "TB/s", "frac": achieved / peak, "sm_mhz": mhz,
-            "peak_source": "measured: cp.async fills of random 512-B rows from L2 alone, "
-                           "115.8 B/clk/SM"}
+            launch(1)
+            launch(2)
+            times = []
+            for r in range(reps):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                launch(3 + r)
+                b.record(stream)
+                torch.cuda.synchronize(device)
+                times.append(a.elapsed_time(b) * 1e-3)
+            ok = int(sink[0].item()) == 0
+            runs.append({"method": ["cp.async", "tma gather4"][method], "warps_per_cta": warps,
+                         "stages": stages, "ctas_per_sm": per_sm,
+                         "tb_per_s": moved / statistics.median(times) / 1e12 if ok else None})
+    best = max((r for r in runs if r["tb_per_s"] is not None), key=lambda r: r["tb_per_s"])
+    return {"tb_per_s": best["tb_per_s"], "best": best, "runs": runs, "row_bytes": row_bytes,
+            "buffer_bytes": PROBE_BUFFER_BYTES, "read_back": True}
 
 
 def _code_only(text: str) -> str:

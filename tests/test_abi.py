@@ -14,12 +14,15 @@ import torch
 import top_sparse_attention_index_b200 as qsa
 from top_sparse_attention_index_b200 import _binding, build_lib
 
-HEADER = Path(__file__).resolve().parent.parent / "include" / "qsa.h"
+INCLUDE = Path(__file__).resolve().parent.parent / "include"
 
 
 def declared_functions():
-    text = re.sub(r"/\*.*?\*/", "", HEADER.read_text(), flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(qsa_\w+)\s*\(", text, flags=re.M)))
+    names = set()
+    for header in sorted(INCLUDE.glob("*.h")):
+        text = re.sub(r"/\*.*?\*/", "", header.read_text(), flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(qsa_\w+)\s*\(", text, flags=re.M))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -320,3 +323,26 @@ def test_shard_ranges():
     assert r[0][0] == 0 and r[-1][1] == 1000
     assert all(lo % 4 == 0 for lo, _ in r) and all(a[1] == b[0] for a, b in zip(r, r[1:]))
     assert qsa.shard_ranges(10, 4, block=4)[-1] == (10, 10)   # more ranks than blocks
+
+
+@pytest.mark.parametrize("over", [
+    dict(method=4), dict(method=-1), dict(read_back=3), dict(row_bytes=128),
+    dict(stages=1), dict(stages=5), dict(warps=0), dict(warps=16), dict(ctas=0), dict(iters=0),
+    dict(pitch=500), dict(pitch=256), dict(src=None), dict(sink=None), dict(src=0x1008),
+    dict(warps=15, stages=4),                      # 480 KiB of shared memory
+])
+def test_probe_rejects_bad_arguments_before_cuda(lib, over):
+    a = dict(method=0, read_back=1, src=0x1000, rows=1024, pitch=512, row_bytes=512, warps=4,
+             stages=2, ctas=8, iters=4, sink=0x2000)
+    a.update(over)
+    st = qsa.qsa_probe_gather(a["method"], a["read_back"], a["src"], a["rows"], a["pitch"],
+                              a["row_bytes"], a["warps"], a["stages"], a["ctas"], a["iters"], 1,
+                              a["sink"], None)
+    assert st == qsa.QSA_ERR_INVALID_ARG, qsa.qsa_last_error_detail()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_probe_valid_arguments_reach_the_device(lib):
+    # without a GPU the first CUDA call fails: the arguments themselves were accepted
+    st = qsa.qsa_probe_gather(1, 1, 0x1000, 1024, 512, 512, 4, 2, 8, 4, 1, 0x2000, None)
+    assert st == qsa.QSA_ERR_CUDA

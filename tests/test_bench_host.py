@@ -92,16 +92,13 @@ def test_kernel_hash_ignores_comments_and_whitespace():
     assert len(bench._kernel_hash()) == 16
 
 
-def test_sm_side_bounds_scale_with_the_sampled_clock():
-    """The shared-memory and L2 bounds are the measured per-SM byte rates times 148 SMs
-    times the sampled clock; the fractions are achieved / peak."""
-    gathered, t = 32.8e9, 2.0e-3
-    for fn, rate in ((bench._smem_bound, bench.GATHER_FILL_WITH_READS_B_PER_CLK),
-                     (bench._l2_bound, bench.GATHER_FILL_ALONE_B_PER_CLK)):
-        r = fn(gathered, t, {"sm_mhz": 1965.0})
-        assert abs(r["peak"] - 148 * rate * 1.965e9 / 1e12) < 1e-9
-        assert abs(r["achieved"] - gathered / t / 1e12) < 1e-9
-        assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
-        slow = fn(gathered, t, {"sm_mhz": 1000.0})
-        assert abs(slow["peak"] / r["peak"] - 1000.0 / 1965.0) < 1e-12
-        assert fn(gathered, t, {"sm_mhz": None})["sm_mhz"] == 1965.0  # unsampled: max clock
+def test_gather_probe_shapes_fit_one_sm():
+    """Every pipeline shape the benchmark's gather probe runs fits the shared memory of one
+    SM at its CTAs per SM (228 KiB, 1 KiB reserved per CTA) and the probe's limits."""
+    for row_bytes, shapes in bench.PROBE_CONFIGS.items():
+        assert row_bytes in (256, 512)
+        for warps, stages, per_sm in shapes:
+            assert 1 <= warps <= 15 and 2 <= stages <= 4 and per_sm >= 1
+            smem = warps * stages * 16 * row_bytes + 2 * warps * stages * 8
+            assert smem <= 227 * 1024
+            assert per_sm * (smem + 1024) <= 228 * 1024

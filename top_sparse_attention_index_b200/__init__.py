@@ -24,6 +24,7 @@ from ._binding import (  # noqa: F401
     qsa_sparse_prefill,
     qsa_sparse_prefill_block,
     qsa_combine_partials,
+    qsa_probe_gather,
     qsa_sparse_prefill_block_plan,
     qsa_sparse_prefill_fp8kv,
     qsa_sparse_prefill_partial,
@@ -44,5 +45,5 @@ __all__ = [
     "qsa_sparse_prefill_partial", "qsa_combine_partials", "sparse_prefill_partial",
     "combine_partials", "sparse_prefill_context_parallel", "shard_ranges",
     "qsa_sparse_prefill_plan", "qsa_sparse_prefill_workspace_bytes", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
-    "load_library", "QSAError",
+    "load_library", "QSAError", "qsa_probe_gather",
 ]

@@ -51,6 +51,8 @@ SIGNATURES = {
     "qsa_sparse_prefill_noalloc": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _f, _p,
                                           _i64, _i64, _i32, _p, _p]),
+    "qsa_probe_gather": (_i32, [_i32, _i32, _p, _i64, _i64, _i32, _i32, _i32, _i32, _i32,
+                                ctypes.c_uint32, _p, _p]),
     "qsa_status_string": (ctypes.c_char_p, [_i32]),
     "qsa_last_error_detail": (ctypes.c_char_p, []),
 }
@@ -115,6 +117,14 @@ def qsa_sparse_prefill_workspace_bytes(Tq, Hq, Hkv, W, D, num_sms) -> int:
         qsa_sparse_prefill_plan(Tq, Hq, Hkv, D, W, num_sms)  # raises with the status
         raise QSAError(QSA_ERR_INVALID_ARG, qsa_last_error_detail())
     return n
+
+
+def qsa_probe_gather(method, read_back, src, rows, pitch_bytes, row_bytes, warps_per_cta, stages,
+                     ctas, iters, seed, sink, stream) -> int:
+    """Raw call of the gather-rate probe (include/qsa_probe.h); returns the status code."""
+    return int(load_library().qsa_probe_gather(method, read_back, src, rows, pitch_bytes,
+                                               row_bytes, warps_per_cta, stages, ctas, iters,
+                                               seed, sink, stream))
 
 
 def qsa_sparse_prefill(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,

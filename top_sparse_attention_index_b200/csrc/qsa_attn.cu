@@ -37,6 +37,7 @@
 // after ldmatrix; Q, P and both MMAs are f16 with fp32 accumulation; k_scale is folded
 // into the softmax scale and v_scale into the final normalisation, so the result is the
 // attention over the dequantised cache up to rounding.
+#include <cuda.h>  // CUtensorMap (the TMA gather's tensor maps)
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -54,10 +55,25 @@ constexpr int kChunks = kRowBytes / 16;     // 32 16-byte chunks per row
 constexpr int kMergeStride = kHeadDim + 4;  // padded fp32 row of the epilogue merge
 constexpr float kNegInf = -__builtin_huge_valf();
 constexpr float kRescaleLog2 = 8.0f;  // lazy-rescale threshold (base-2 exponent)
+constexpr uint32_t kMaxPolls = 1u << 20;  // bound of one mbarrier wait (TMA gathers)
+// E4M3 shapes with this many slot lanes read all of a warp's V code pairs early (the
+// eight-CTA shape of one lane: 1.482 vs 1.489 ms with two pairs)
+#ifndef QSA_FP8_EARLY_ALL_LANES
+#define QSA_FP8_EARLY_ALL_LANES 1
+#endif
 
+
+// Tensor maps of the TMA gather, one per KV head for K and for V: a 2-D view [S rows,
+// 256 elements] of that head's slice of the cache (row pitch = the slot stride), a box of
+// one 128-byte column block of one row, 128-byte swizzle (tile::gather4 row gathers).
+constexpr int kMaxTmaHeads = 4;
+struct TmaMaps {
+  CUtensorMap k[kMaxTmaHeads];
+  CUtensorMap v[kMaxTmaHeads];
+};
 
 template <int NTILE, int DSPLIT, int SL, int STAGES, bool KV8 = false, bool SLOT16 = false,
-          int QROWS = NTILE * 8>
+          int QROWS = NTILE * 8, bool TMA = false>
 struct Cfg {
   // warps serving one slot lane: a D-split pair (each warp handles every head tile over
   // its half of D) or one warp per head tile
@@ -86,8 +102,18 @@ struct Cfg {
   // registers
   static constexpr bool kXchgOverQ = DSPLIT > 1;
   static_assert(!kXchgOverQ || kXchgBytes <= kQBytes, "exchange buffer fits the Q tile");
-  static constexpr size_t kSmem =
-      size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes + (kXchgOverQ ? 0 : kXchgBytes);
+  // TMA gathers: one full barrier per (slot lane, stage), after the scan words
+  static_assert(!TMA || DSPLIT == 2, "the TMA gather serves the D-split pair shapes");
+  static constexpr int kBarBytes = TMA ? SL * STAGES * 8 : 0;
+  static constexpr size_t kSmem = size_t(kRingBytes) + kQBytes + kIdxBytes + kScanBytes +
+                                  (kXchgOverQ ? 0 : kXchgBytes) + kBarBytes;
+  // Layout of a gathered sub-tile in shared memory.  cp.async: 16 rows of kKvRow bytes,
+  // 16-byte chunk c of row r at r * kKvRow + ((c ^ (r & 7)) << 4).  TMA tile::gather4
+  // (128-byte swizzle): kKvRow / 128 column blocks of [16 rows x 128 bytes], chunk c of
+  // row r at (c / 8) * 2048 + r * 128 + (((c % 8) ^ (r & 7)) << 4).  Both are the same
+  // XOR of the chunk's low three bits; only the row and block pitches differ.
+  static constexpr int kRowPitch = TMA ? 128 : kKvRow;
+  static constexpr int kBlkPitch = TMA ? 16 * 128 : 128;
   // the epilogue's merge buffer reuses the ring and, after it, the Q tile and the slot
   // list (all dead once the main loop is over)
   static_assert(kMergeBytes <= kRingBytes + kQBytes + kIdxBytes, "merge buffer fits");
@@ -109,12 +135,12 @@ struct Cfg {
 // ldmatrix delivers for 8-bit data; a sum over D does not depend on that order, and the
 // epilogue maps the m-tile rows back.
 template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8, bool SLOT16,
-          int QROWS>
+          int QROWS, bool TMA>
 __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
-    qsa_sparse_attn_fwd_kernel(const FwdParams p) {
+    qsa_sparse_attn_fwd_kernel(const FwdParams p, const __grid_constant__ TmaMaps maps) {
   static_assert(!QSPLIT || DSPLIT == 2, "splitting Q K^T needs a D-split pair");
   constexpr int kKS = QSPLIT ? 8 : 16;  // k-steps of Q K^T per warp
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16, QROWS>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16, QROWS, TMA>;
   using SlotT = std::conditional_t<SLOT16, uint16_t, uint32_t>;
   constexpr int kKvRow = C::kKvRow;
   constexpr int kMT = 16 / DSPLIT;  // m16 tiles of D per warp in the PV product
@@ -127,6 +153,10 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   int32_t* sScan = reinterpret_cast<int32_t*>(sSlot + kMaxSlotsPerSplit);
   float4* sXchg = C::kXchgOverQ ? reinterpret_cast<float4*>(sQ)  // (QSPLIT only)
                                  : reinterpret_cast<float4*>(sScan + 32);
+  // TMA: full barrier of (slot lane, stage); both warps of the lane's pair arrive on it
+  // with the byte count of their half of the sub-tile
+  uint64_t* sBar = reinterpret_cast<uint64_t*>(sScan + 32);
+  auto full_bar = [&](int lane_i, int stage) { return smem_addr(sBar + lane_i * STAGES + stage); };
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -155,6 +185,18 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
       wv = wv < 0 ? 0 : p.W;
     }
     width_t = wv;
+  }
+  if constexpr (TMA) {
+    // the 128-byte swizzle of the TMA destinations repeats every 1024 bytes: the ring must
+    // start on that boundary (it does with no static shared memory; checked, not assumed)
+    if ((smem_addr(smem) & 1023u) != 0) {
+      if (tid == 0 && p.err_word != nullptr) atomicOr(p.err_word, 8u);
+      return;
+    }
+    if (tid == 0) {
+      for (int i = 0; i < SL * STAGES; ++i) mbar_init(smem_addr(sBar + i), C::kParts);
+      mbar_init_fence();
+    }
   }
   // ---- 0. the group's Q rows (commit group 0): in flight during the index work ---------
   const int G = p.G;
@@ -288,7 +330,31 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
         sl[0] = s4.x; sl[1] = s4.y; sl[2] = s4.z; sl[3] = s4.w;
       }
     };
-    if constexpr (!KV8) {
+    if constexpr (TMA) {
+      // each warp of the pair gathers its rows of K and V with TMA tile::gather4 (four
+      // rows of one 128-byte column block per instruction), one instruction per lane, all
+      // issued at once; lane 0 first announces the warp's bytes on the stage's full
+      // barrier (which expects both warps of the pair)
+      constexpr int kBlk = kKvRow / 128;
+      constexpr int kBoxElems = KV8 ? 128 : 64;
+      constexpr int kIssue = (kLoadRows / 4) * kBlk * 2;  // (row group, block, K or V)
+      static_assert(kIssue <= 32, "one gather4 per lane");
+      const uint32_t bar = full_bar(wslot, buf);
+      if (lane == 0) mbar_arrive_expect_tx(bar, kLoadRows * kKvRow * 2);
+      __syncwarp();
+      if (lane < kIssue) {
+        const int tv = lane & 1;               // 0: K, 1: V
+        const int b = (lane >> 1) % kBlk;      // column block
+        const int gi = (lane >> 1) / kBlk;     // row group of the warp's rows
+        uint32_t sl[4];
+        slots4(4 * gi, sl);
+        const uint32_t d = sub_s + buf * C::kSubBytes + (row0 + 4 * gi) * C::kRowPitch +
+                           b * C::kBlkPitch + tv * 16 * kKvRow;
+        fence_proxy_async_smem();  // the pair's earlier reads of this buffer come first
+        tma_gather4(d, tv ? &maps.v[j] : &maps.k[j], bar, b * kBoxElems, int32_t(sl[0]),
+                    int32_t(sl[1]), int32_t(sl[2]), int32_t(sl[3]));
+      }
+    } else if constexpr (!KV8) {
       uint32_t kd[8];
 #pragma unroll
       for (int m = 0; m < 8; ++m) kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (m << 4));
@@ -409,7 +475,8 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   // ldmatrix addressing.  Chunk c of a row sits at ((c ^ key) << 4), key = row & 7 =
   // lane & 7 for every row this lane addresses.  With c = 2 * step + hi (step = k-step
   // for K, m-tile for V; hi in {0, 1}) the XOR only touches the low three bits, so
-  // (c ^ key) << 4 = 128 * (step >> 2) + swz[step & 3]: four per-lane offsets computed
+  // (c ^ key) << 4 = 128 * (step >> 2) + swz[step & 3] (128 is the block pitch kBlkPitch
+  // of the cp.async layout; the TMA layout has 2048): four per-lane offsets computed
   // once, and every ldmatrix address in the loop is a register plus an immediate.
   const int key = lane & 7;
   const int krow = (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -419,12 +486,13 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   uint32_t kswz[4], vswz[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    kswz[m] = uint32_t(krow * kKvRow + (((2 * m + khi) ^ key) << 4));
+    kswz[m] = uint32_t(krow * C::kRowPitch + (((2 * m + khi) ^ key) << 4));
     // E4M3 V: the transposed loads use the K lane pattern (one chunk is one m-tile)
     vswz[m] = KV8 ? kswz[m] + 16 * kKvRow
-                  : uint32_t(16 * kRowBytes + vrow * kRowBytes + (((2 * m + vhi) ^ key) << 4));
+                  : uint32_t(16 * kRowBytes + vrow * C::kRowPitch + (((2 * m + vhi) ^ key) << 4));
   }
   const float sl2 = p.scale_log2;
+  bool tma_failed = false;
 
   for (int s = 0; s < n_stages; ++s) {
     cp_async_wait<STAGES - 2>();
@@ -438,12 +506,20 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     const int base = s * C::kRows + wslot * 16;
     if (base >= n_valid) continue;  // warp-uniform: no valid slot in this sub-tile
     const uint32_t sub = sub_s + buf * C::kSubBytes;
+    if constexpr (TMA) {
+      // the stage's K and V rows of both warps have landed (use s / STAGES of the buffer);
+      // a bounded wait: on a time-out the error bit is set, later waits are skipped and
+      // the rows' outputs are not valid, but no warp leaves the pair's barriers
+      if (!tma_failed && !mbar_wait(full_bar(wslot, buf), (s / STAGES) & 1, kMaxPolls))
+        tma_failed = true;
+    }
 
     // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8) per head tile; each K
     // fragment feeds every tile of the warp; two chains for ILP.
     uint32_t kt[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) kt[m] = sub + kswz[m] + ks0 * (KV8 ? 16 : 32);  // a k-step's bytes
+    for (int m = 0; m < 4; ++m)  // a k-step is 32 (16) bytes of a row: whole 128-byte blocks
+      kt[m] = sub + kswz[m] + (ks0 * (KV8 ? 16 : 32) / 128) * C::kBlkPitch;
     float sa[TPW][4], sb[TPW][4];
 #pragma unroll
     for (int nt = 0; nt < TPW; ++nt)
@@ -453,10 +529,10 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
 #pragma unroll
       for (int ks = 0; ks < kKS; ks += 2) {
         uint32_t a[4];
-        ldmatrix_x4(a, kt[ks & 3] + 128 * (ks >> 2));
+        ldmatrix_x4(a, kt[ks & 3] + C::kBlkPitch * (ks >> 2));
 #pragma unroll
         for (int nt = 0; nt < TPW; ++nt) mma_bf16_16816(sa[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
-        ldmatrix_x4(a, kt[(ks + 1) & 3] + 128 * ((ks + 1) >> 2));
+        ldmatrix_x4(a, kt[(ks + 1) & 3] + C::kBlkPitch * ((ks + 1) >> 2));
 #pragma unroll
         for (int nt = 0; nt < TPW; ++nt)
           mma_bf16_16816(sb[nt], a, qf[nt][ks + 1][0], qf[nt][ks + 1][1]);
@@ -467,7 +543,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
 #pragma unroll
       for (int kq = 0; kq < kKS / 2; ++kq) {
         uint32_t r[4], a[4];
-        ldmatrix_x4(r, kt[kq & 3] + 128 * (kq >> 2));
+        ldmatrix_x4(r, kt[kq & 3] + C::kBlkPitch * (kq >> 2));
         e4m3x4_to_f16x2x2(r[0], a[0], a[2]);
         e4m3x4_to_f16x2x2(r[1], a[1], a[3]);
 #pragma unroll
@@ -488,17 +564,17 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     // With one head tile per warp the first kVEarly V fragments of the sub-tile (bf16: m-tiles;
     // E4M3: raw codes of m-tile pairs) are read here, before the score exchange and the
     // softmax, so their shared-memory latency is hidden behind that work (the stage has
-    // landed; the registers fit under the cap).  The E4M3 shape of two slot lanes has the
-    // registers for all of its pairs (measured 1.738 vs 1.759 ms).  With two head tiles per
+    // landed; the registers fit under the cap).  The E4M3 shape of one slot lane has the
+    // registers for all of its pairs.  With two head tiles per
     // warp the registers are already at the cap and the early reads cost more than they hide.
-    constexpr int kVEarly = TPW == 1 ? (KV8 ? (SL == 2 ? kMT / 2 : 2) : 4) : 0;
+    constexpr int kVEarly = TPW == 1 ? (KV8 ? (SL == QSA_FP8_EARLY_ALL_LANES ? kMT / 2 : 2) : 4) : 0;
     uint32_t vt[4];
     uint32_t vearly[kVEarly > 0 ? kVEarly : 1][4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / (KV8 ? 8 : 4)) * 128;
+    for (int m = 0; m < 4; ++m) vt[m] = sub + vswz[m] + wd * (kMT / (KV8 ? 8 : 4)) * C::kBlkPitch;
 #pragma unroll
     for (int mt = 0; mt < kVEarly; ++mt)
-      ldmatrix_x4_trans(vearly[mt], vt[mt & 3] + 128 * (mt >> 2));
+      ldmatrix_x4_trans(vearly[mt], vt[mt & 3] + C::kBlkPitch * (mt >> 2));
     if constexpr (QSPLIT) {
       // each warp of the pair holds the scores over its half of D: exchange and add in
       // a fixed order (low half + high half) so both warps hold the same scores
@@ -600,7 +676,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
         if (mt < kVEarly) {
           a[0] = vearly[mt][0]; a[1] = vearly[mt][1]; a[2] = vearly[mt][2]; a[3] = vearly[mt][3];
         } else {
-          ldmatrix_x4_trans(a, vt[mt & 3] + 128 * (mt >> 2));
+          ldmatrix_x4_trans(a, vt[mt & 3] + C::kBlkPitch * (mt >> 2));
         }
 #pragma unroll
         for (int nt = 0; nt < TPW; ++nt) mma_bf16_16816(o[nt][mt], a, b0[nt], b1[nt]);
@@ -616,7 +692,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
         if (mq < kVEarly) {
           r[0] = vearly[mq][0]; r[1] = vearly[mq][1]; r[2] = vearly[mq][2]; r[3] = vearly[mq][3];
         } else {
-          ldmatrix_x4_trans(r, vt[mq & 3] + 128 * (mq >> 2));
+          ldmatrix_x4_trans(r, vt[mq & 3] + C::kBlkPitch * (mq >> 2));
         }
         e4m3x4_to_f16x2x2(byte_perm(r[0], 0u, 0x3120u), a[0], a[1]);
         e4m3x4_to_f16x2x2(byte_perm(r[1], 0u, 0x3120u), a[2], a[3]);
@@ -630,6 +706,15 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     }
   }
   cp_async_wait<0>();
+  if constexpr (TMA) {
+    if (tma_failed) {
+      // bounded drain of this lane's gathers that may still be in flight, then report
+      const int lane_stages = n_valid > wslot * 16 ? (n_valid - wslot * 16 + C::kRows - 1) / C::kRows : 0;
+      for (int s = lane_stages > STAGES ? lane_stages - STAGES : 0; s < lane_stages; ++s)
+        mbar_wait(full_bar(wslot, s % STAGES), (s / STAGES) & 1, kMaxPolls / 64);
+      if (lane == 0 && p.err_word != nullptr) atomicOr(p.err_word, 8u);
+    }
+  }
   __syncthreads();  // every warp is done with the ring: reuse it for the merge
 
   // ---- 4. merge the warps of each n8 tile and write ------------------------------------
@@ -783,12 +868,27 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
 }
 
 template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8,
-          bool SLOT16 = false, int QROWS = NTILE * 8>
+          bool SLOT16 = false, int QROWS = NTILE * 8, bool TMA = false>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
-  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16, QROWS>;
+  using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16, QROWS, TMA>;
   if (p.G > QROWS) return cudaErrorInvalidValue;  // the Q tile holds the whole group
   auto kern =
-      qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16, QROWS>;
+      qsa_sparse_attn_fwd_kernel<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16, QROWS, TMA>;
+  TmaMaps maps{};
+  if constexpr (TMA) {
+    if (p.Hkv > kMaxTmaHeads || p.S <= 0) return cudaErrorInvalidValue;
+    const int64_t elem = KV8 ? 1 : 2;
+    for (int jh = 0; jh < p.Hkv; ++jh) {
+      cudaError_t e = encode_row_gather_map(
+          &maps.k[jh], static_cast<const uint8_t*>(p.k_cache) + jh * p.k_stride_h * elem,
+          uint64_t(p.S), uint32_t(kHeadDim * elem), p.k_row_bytes);
+      if (e == cudaSuccess)
+        e = encode_row_gather_map(
+            &maps.v[jh], static_cast<const uint8_t*>(p.v_cache) + jh * p.v_stride_h * elem,
+            uint64_t(p.S), uint32_t(kHeadDim * elem), p.v_row_bytes);
+      if (e != cudaSuccess) return e;
+    }
+  }
   // The shared-memory opt-in is a function attribute that lives in the CUDA context: set
   // it on the first launch in each context only (keyed by the context's unique ID, so a
   // device reset or a new context sets it again), so later calls (e.g. under stream
@@ -809,8 +909,31 @@ cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
     if (dev >= 0 && dev < 64 && now != 0) configured_ctx[dev].store(now, std::memory_order_release);
   }
   const unsigned grid = static_cast<unsigned>(int64_t(p.Tq) * p.Hkv * p.nsplit);
-  kern<<<grid, C::kThreads, C::kSmem, stream>>>(p);
+  kern<<<grid, C::kThreads, C::kSmem, stream>>>(p, maps);
   return cudaGetLastError();
+}
+
+// The same shape with the rows gathered by TMA tile::gather4 (use_tma) or by cp.async.
+// Gather of the K / V rows per cache format: TMA tile::gather4 (1) or cp.async (0).
+// Measured on the long prefill (bf16 2.03 vs 3.10 ms, E4M3 1.74 vs 2.56 ms, G = 12 4.52 vs
+// 6.53 ms): cp.async for both; the TMA kernels stay buildable for measurement.
+#ifndef QSA_TMA_E4M3
+#define QSA_TMA_E4M3 0
+#endif
+#ifndef QSA_TMA_BF16
+#define QSA_TMA_BF16 0
+#endif
+
+// (The TMA kernels are only compiled in when a build asks for them.)
+template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8,
+          bool SLOT16 = false, int QROWS = NTILE * 8>
+cudaError_t launch_gather(const FwdParams& p, cudaStream_t stream, bool use_tma) {
+  if constexpr ((KV8 && QSA_TMA_E4M3) || (!KV8 && QSA_TMA_BF16)) {
+    if (use_tma)
+      return launch_fwd<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16, QROWS, true>(p,
+                                                                                          stream);
+  }
+  return launch_fwd<NTILE, DSPLIT, SL, STAGES, MINB, QSPLIT, KV8, SLOT16, QROWS, false>(p, stream);
 }
 
 // The two shapes (slot lanes x pipeline stages per lane x resident CTAs per SM, chosen by
@@ -875,9 +998,9 @@ static_assert(CfgLarge8::kSmem <= CfgLarge8::kSmPerCta(QSA_LARGE_CTAS), "E4M3 la
 // better than two CTAs of three lanes (measured: long prefill 2.016 vs 2.096 ms, 512-slot
 // rows 0.317 vs 0.356 ms).  A CTA of two lanes takes ~1.4x as long per unit, so with few
 // units the coarser waves lose (4,000 units: 0.557 vs 0.564 ms; 2,048: 0.303 vs 0.297;
-// 512: 140 vs 102 us): the shape is used from eight of its waves on.  E4M3 caches do the
-// same with two slot lanes of four stages (long prefill 1.756 vs 1.789 ms; with fewer waves
-// they keep four lanes of three stages, with the 16-bit list).
+// 512: 140 vs 102 us): the shape is used from eight waves of three CTAs per SM on.  E4M3
+// caches take a shape of their own there (below; with fewer waves they keep four lanes of
+// three stages, with the 16-bit list).
 constexpr int64_t kRows16 = 65536;
 constexpr int64_t kShape16MinWaves = 8;
 #ifndef QSA_SMALL16_SL
@@ -889,17 +1012,26 @@ constexpr int64_t kShape16MinWaves = 8;
 #ifndef QSA_SMALL16_CTAS
 #define QSA_SMALL16_CTAS 3
 #endif
+// E4M3 caches in such launches: one slot lane (a warp pair) of two stages, 25 KB, eight
+// CTAs per SM (long prefill 1.495 ms; two lanes of two stages at three or four CTAs 1.595,
+// of four stages 1.738; one lane of three stages at six CTAs 1.684, of four at five 1.749)
 #ifndef QSA_FP8_SMALL16_SL
-#define QSA_FP8_SMALL16_SL 2
+#define QSA_FP8_SMALL16_SL 1
 #endif
 #ifndef QSA_FP8_SMALL16_STAGES
-#define QSA_FP8_SMALL16_STAGES 4
+#define QSA_FP8_SMALL16_STAGES 2
+#endif
+#ifndef QSA_FP8_SMALL16_CTAS
+#define QSA_FP8_SMALL16_CTAS 8
+#endif
+#ifndef QSA_LARGE16_CTAS
+#define QSA_LARGE16_CTAS 3
 #endif
 using CfgSmall16 = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES, false, true>;
 using CfgSmall8r16 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true, true>;
 using CfgSmall8s16 = Cfg<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES, true, true>;
 static_assert(CfgSmall16::kSmem <= CfgSmall16::kSmPerCta(QSA_SMALL16_CTAS), "16-bit shape: CTAs per SM");
-static_assert(CfgSmall8s16::kSmem <= CfgSmall8s16::kSmPerCta(QSA_SMALL16_CTAS),
+static_assert(CfgSmall8s16::kSmem <= CfgSmall8s16::kSmPerCta(QSA_FP8_SMALL16_CTAS),
               "E4M3 three-CTA shape: CTAs per SM");
 // 8 < G <= 12 on such caches: two slot lanes of two stages with a 12-row Q tile, three CTAs
 // per SM (G = 12: 2.518 vs 2.609 ms for 8,000 query rows of a 12,288-slot cache, 1.289 vs
@@ -914,7 +1046,7 @@ static_assert(CfgSmall8s16::kSmem <= CfgSmall8s16::kSmPerCta(QSA_SMALL16_CTAS),
 #define QSA_LARGE16_QROWS 12
 #endif
 using CfgLarge16 = Cfg<2, 2, QSA_LARGE16_SL, QSA_LARGE16_STAGES, false, true, QSA_LARGE16_QROWS>;
-static_assert(CfgLarge16::kSmem <= CfgLarge16::kSmPerCta(QSA_SMALL16_CTAS),
+static_assert(CfgLarge16::kSmem <= CfgLarge16::kSmPerCta(QSA_LARGE16_CTAS),
               "12-row two-tile shape: CTAs per SM");
 static_assert(CfgSmall8r16::kSmem <= CfgSmall8r16::kSmPerCta(QSA_SMALL_CTAS),
               "E4M3 16-bit shape: CTAs per SM");
@@ -949,27 +1081,38 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   const bool rows16 = p.S <= kRows16;
   const int64_t grid = int64_t(p.Tq) * p.Hkv * p.nsplit;
   const bool shape16 =
-      rows16 && p.num_sms > 0 && grid >= kShape16MinWaves * p.num_sms * QSA_SMALL16_CTAS;
+      rows16 && p.num_sms > 0 && grid >= kShape16MinWaves * p.num_sms * 3;
+  // TMA tile::gather4 for the rows where it is the faster gather (per cache format; one
+  // tensor map per KV head for K and V, so at most kMaxTmaHeads heads; an empty shard
+  // (S == 0) gathers nothing and takes the cp.async kernel)
+  const bool tma_shape = p.S > 0 && p.Hkv <= kMaxTmaHeads;
+  const bool tma = tma_shape && (p.kv_fp8 ? QSA_TMA_E4M3 : QSA_TMA_BF16);
   if (p.kv_fp8) {
     if (p.G <= 8)
-      e = shape16 ? launch_fwd<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES, QSA_SMALL16_CTAS,
-                               true, true, true>(p, stream)
-          : rows16 ? launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
-                                true, true>(p, stream)
-                   : launch_fwd<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS, true,
-                                true>(p, stream);
+      e = shape16 ? launch_gather<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES,
+                                  QSA_FP8_SMALL16_CTAS, true, true, true>(p, stream, tma)
+          : rows16 ? launch_gather<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS,
+                                   true, true, true>(p, stream, tma)
+                   : launch_gather<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS,
+                                   true, true>(p, stream, tma);
+    else if constexpr (QSA_LARGE_DSPLIT == 2)
+      e = launch_gather<2, 2, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, QSA_LARGE_CTAS, true,
+                        true>(p, stream, tma);
     else
       e = launch_fwd<2, QSA_LARGE_DSPLIT, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, QSA_LARGE_CTAS,
                      kLargeQsplit, true>(p, stream);
   } else {
     if (p.G <= 8)
-      e = shape16 ? launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES,
-                               QSA_SMALL16_CTAS, QSA_SMALL_QSPLIT, false, true>(p, stream)
-                  : launch_fwd<1, QSA_SMALL_DSPLIT, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
-                               QSA_SMALL_QSPLIT, false>(p, stream);
+      e = shape16 ? launch_gather<1, 2, QSA_SMALL16_SL, QSA_SMALL16_STAGES, QSA_SMALL16_CTAS,
+                                  QSA_SMALL_QSPLIT, false, true>(p, stream, tma)
+                  : launch_gather<1, 2, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
+                                  QSA_SMALL_QSPLIT, false>(p, stream, tma);
     else if (shape16 && p.G <= QSA_LARGE16_QROWS)
-      e = launch_fwd<2, 2, QSA_LARGE16_SL, QSA_LARGE16_STAGES, QSA_SMALL16_CTAS, true, false, true,
-                     QSA_LARGE16_QROWS>(p, stream);
+      e = launch_gather<2, 2, QSA_LARGE16_SL, QSA_LARGE16_STAGES, QSA_LARGE16_CTAS, true, false,
+                        true, QSA_LARGE16_QROWS>(p, stream, tma);
+    else if constexpr (QSA_LARGE_DSPLIT == 2)
+      e = launch_gather<2, 2, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS, true, false>(
+          p, stream, tma);
     else
       e = launch_fwd<2, QSA_LARGE_DSPLIT, QSA_LARGE_SL, QSA_LARGE_STAGES, QSA_LARGE_CTAS,
                      kLargeQsplit, false>(p, stream);

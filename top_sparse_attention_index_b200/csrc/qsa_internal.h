@@ -2,6 +2,7 @@
 // kernels (qsa_attn.cu).  Not installed; not part of the public ABI.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -102,6 +103,12 @@ void set_error_detail(const char* fmt, ...);
 // attributes) is cached under this ID, so a device reset or a new primary context
 // invalidates the cache instead of leaving stale addresses behind.
 uint64_t current_context_id();
+
+// 2-D tensor map over `rows` rows of `row_bytes` bytes (512: bf16, 256: E4M3 codes),
+// `pitch` bytes apart, for tile::gather4 row gathers: a box of one 128-byte column block
+// of one row, 128-byte swizzle.  Host only (the driver's encoder, looked up once).
+cudaError_t encode_row_gather_map(CUtensorMap* map, const void* base, uint64_t rows,
+                                  uint32_t row_bytes, uint64_t pitch);
 size_t workspace_lse_offset(int32_t Tq, int32_t Hq, int32_t nsplit);
 
 }  // namespace qsa

@@ -239,17 +239,22 @@ qsa_status_t qsa_sparse_prefill_fp8kv(const void* q, int64_t q_stride_t, int64_t
  *   S_total            global slot extent (>= slot_lo + S).  Selected entries in
  *                      [0, S_total) outside this device's range are skipped silently;
  *                      entries outside [-1, S_total) set QSA_ERRBIT_SLOT_RANGE.
- *   part_o             fp32 [Tq, Hq, D] contiguous (16-byte aligned): the output
- *                      normalised over this device's valid slots (zeros where it has none).
+ *   part_o             [Tq, Hq, D] contiguous (16-byte aligned), fp32 or, with
+ *                      record_bf16 = 1, bf16 (round to nearest even; half the bytes to
+ *                      exchange): the output normalised over this device's valid slots
+ *                      (zeros where it has none).
  *   part_lse           fp32 [Tq, Hq] contiguous: log2 of the sum over this device's valid
  *                      slots of 2^(scale * log2(e) * s_i) (k_scale included for E4M3), i.e.
  *                      the base-2 log-sum-exp of the scaled scores; -inf where none.
+ *                      Always fp32.
+ *   record_bf16        0: part_o fp32; 1: part_o bf16.  Any other value: QSA_ERR_INVALID_ARG.
  * The split plan and workspace are those of qsa_sparse_prefill_block_plan; the device's
  * own splits are combined into the one record before the call's work ends.
  *
  * qsa_combine_partials: out[t, h, :] = sum_r 2^(lse_r - m) O_r / sum_r 2^(lse_r - m),
- * m = max_r lse_r, over R records stacked as part_o [R, Tq, Hq, D] and part_lse
- * [R, Tq, Hq] (the layout an all-gather of the records produces); records with
+ * m = max_r lse_r, over R records stacked as part_o [R, Tq, Hq, D] (fp32, or bf16 with
+ * record_bf16 = 1) and part_lse fp32 [R, Tq, Hq] (the layout an all-gather of the
+ * records produces); the sums run in fp32 in record order; records with
  * lse = -inf weigh 0; a row with no record above -inf is written as exact zeros.  out is
  * bf16 [Tq, Hq, D] with strides (out_stride_t, out_stride_h, 1), multiples of 8.
  * Both entry points enqueue on `stream` only and allocate nothing.
@@ -262,12 +267,13 @@ qsa_status_t qsa_sparse_prefill_partial(const void* q, int64_t q_stride_t, int64
                                         const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
                                         int32_t D, int64_t S, int32_t W, int32_t block,
                                         int64_t slot_lo, int64_t S_total, int32_t kv_fp8,
-                                        float scale, float k_scale, float v_scale, float* part_o,
-                                        float* part_lse, int32_t nsplit, void* workspace,
-                                        size_t workspace_bytes, uint32_t* err_word, void* stream);
+                                        float scale, float k_scale, float v_scale, void* part_o,
+                                        float* part_lse, int32_t record_bf16, int32_t nsplit,
+                                        void* workspace, size_t workspace_bytes,
+                                        uint32_t* err_word, void* stream);
 
-qsa_status_t qsa_combine_partials(const float* part_o, const float* part_lse, int32_t R,
-                                  int32_t Tq, int32_t Hq, int32_t D, void* out,
+qsa_status_t qsa_combine_partials(const void* part_o, const float* part_lse, int32_t record_bf16,
+                                  int32_t R, int32_t Tq, int32_t Hq, int32_t D, void* out,
                                   int64_t out_stride_t, int64_t out_stride_h, void* stream);
 
 /* Size of the device scratch array that qsa_sparse_prefill_noalloc uses (16 MiB). */

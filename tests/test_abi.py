@@ -50,7 +50,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_status_strings(lib):
-    assert qsa.qsa_abi_version() == 1
+    assert qsa.qsa_abi_version() == 2
     for code, name in [(0, "QSA_OK"), (1, "QSA_ERR_INVALID_ARG"), (2, "QSA_ERR_UNSUPPORTED"),
                        (3, "QSA_ERR_WORKSPACE"), (4, "QSA_ERR_CUDA")]:
         assert qsa.qsa_status_string(code) == name
@@ -266,8 +266,8 @@ def _call_partial(**over):
              k_stride_h=256, v_cache=0x30000, v_stride_s=512, v_stride_h=256, slot_idx=0x40000,
              idx_stride_t=8, width=None, Tq=4, Hq=16, Hkv=2, D=256, S=100, W=8, block=1,
              slot_lo=0, S_total=100, kv_fp8=0, scale=0.0625, k_scale=1.0, v_scale=1.0,
-             part_o=0x50000, part_lse=0x60000, nsplit=1, workspace=None, workspace_bytes=0,
-             err_word=None, stream=None)
+             part_o=0x50000, part_lse=0x60000, record_bf16=0, nsplit=1, workspace=None,
+             workspace_bytes=0, err_word=None, stream=None)
     a.update(over)
     return qsa.qsa_sparse_prefill_partial(**a)
 
@@ -281,6 +281,8 @@ INVALID_PARTIAL = [
     (dict(slot_lo=50, S_total=120), qsa.QSA_ERR_INVALID_ARG),  # S_total < slot_lo + S
     (dict(S_total=-1), qsa.QSA_ERR_INVALID_ARG),
     (dict(kv_fp8=2), qsa.QSA_ERR_INVALID_ARG),
+    (dict(record_bf16=2), qsa.QSA_ERR_INVALID_ARG),
+    (dict(record_bf16=-1), qsa.QSA_ERR_INVALID_ARG),
     (dict(D=128), qsa.QSA_ERR_UNSUPPORTED),
     (dict(k_cache=None), qsa.QSA_ERR_INVALID_ARG),            # S > 0 needs the caches
 ]
@@ -306,15 +308,16 @@ def test_partial_valid_shard_reaches_the_device_query(lib):
 @pytest.mark.skipif(torch.cuda.is_available(),
                     reason="fake-pointer validation runs only where no GPU can be reached")
 def test_combine_partials_validation(lib):
-    ok = dict(part_o=0x50000, part_lse=0x60000, R=2, Tq=4, Hq=16, D=256, out=0x70000,
-              out_stride_t=16 * 256, out_stride_h=256, stream=None)
+    ok = dict(part_o=0x50000, part_lse=0x60000, record_bf16=0, R=2, Tq=4, Hq=16, D=256,
+              out=0x70000, out_stride_t=16 * 256, out_stride_h=256, stream=None)
     bad = [dict(R=0), dict(Hq=0), dict(Tq=-1), dict(part_o=None), dict(out=None),
-           dict(part_o=0x50008), dict(out_stride_h=12)]
+           dict(part_o=0x50008), dict(out_stride_h=12), dict(record_bf16=2)]
     for over in bad:
         assert qsa.qsa_combine_partials(**{**ok, **over}) == qsa.QSA_ERR_INVALID_ARG, over
     assert qsa.qsa_combine_partials(**{**ok, "D": 128}) == qsa.QSA_ERR_UNSUPPORTED
     assert qsa.qsa_combine_partials(**{**ok, "Tq": 0, "part_o": None}) == qsa.QSA_OK
     assert qsa.qsa_combine_partials(**ok) == qsa.QSA_ERR_CUDA   # valid: the launch fails
+    assert qsa.qsa_combine_partials(**{**ok, "record_bf16": 1}) == qsa.QSA_ERR_CUDA
 
 
 def test_shard_ranges():

@@ -41,8 +41,9 @@ def _case():
 
 
 def _partial_double(q, k_local, v_local, slot_idx, slot_lo, S_total, width=None, scale=None,
-                    block=1, k_scale=1.0, v_scale=1.0):
-    """float64 restatement of qsa_sparse_prefill_partial's documented record."""
+                    block=1, k_scale=1.0, v_scale=1.0, record_dtype=torch.float32):
+    """float64 restatement of qsa_sparse_prefill_partial's documented record (the
+    normalised output rounded to record_dtype, the log-sum-exp in fp32)."""
     scale = 1.0 / 16.0 if scale is None else scale
     Tq, Hq, _ = q.shape
     S_loc, Hkv, _ = k_local.shape
@@ -60,7 +61,7 @@ def _partial_double(q, k_local, v_local, slot_idx, slot_lo, S_total, width=None,
             p = np.exp2(x - m)
             o[t, h] = (p @ vd[sel, h // G]) / p.sum()
             lse[t, h] = m + math.log2(p.sum())
-    return torch.from_numpy(o), torch.from_numpy(lse)
+    return torch.from_numpy(o).to(record_dtype), torch.from_numpy(lse)
 
 
 def _combine_double(g_o, g_l, out=None):
@@ -72,7 +73,7 @@ def _combine_double(g_o, g_l, out=None):
     return torch.from_numpy(np.where(den[..., None] > 0, num / np.maximum(den, 1e-300)[..., None], 0.0))
 
 
-def _rank_main(rank, world, port, queue):
+def _rank_main(rank, world, port, queue, record_dtype):
     import torch.distributed as dist
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -83,7 +84,8 @@ def _rank_main(rank, world, port, queue):
     lo, hi = cp.shard_ranges(S, world)[rank]
     out = cp.sparse_prefill_context_parallel(q, k[lo:hi], v[lo:hi], idx, lo, S,
                                              partial_fn=_partial_double,
-                                             combine_fn=_combine_double)
+                                             combine_fn=_combine_double,
+                                             record_dtype=record_dtype)
     queue.put((rank, out.numpy()))
     dist.barrier()
     dist.destroy_process_group()
@@ -95,11 +97,12 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _run(world):
+def _run(world, record_dtype=torch.float32):
     ctx = mp.get_context("spawn")
     queue = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, queue)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, queue, record_dtype))
+             for r in range(world)]
     for p in procs:
         p.start()
     results = dict(queue.get(timeout=180) for _ in procs)
@@ -117,6 +120,22 @@ def test_context_parallel_exchange_matches_the_whole_cache(oracle_lib):
         for r in range(world):
             np.testing.assert_allclose(results[r], ref, rtol=1e-5, atol=1e-6)
         assert np.all(results[0][1] == 0)   # the fully masked row
+
+
+def test_context_parallel_bf16_records(oracle_lib):
+    """bf16 records: every record's normalised output is rounded to bf16 (relative error at
+    most 2^-9) and the combine is a convex combination of the records, so the result is
+    within 2^-9 of the largest |V| element of the row's selected rows of the whole-cache
+    oracle (here bounded by the largest |V| of the cache)."""
+    q, k, v, idx = _case()
+    ref = oracle_lib.forward(q, k, v, idx, None, 1.0 / 16.0)
+    bound = 2.0 ** -9 * float(v.float().abs().max()) + 1e-6
+    for world in (2, 3):
+        results = _run(world, torch.bfloat16)
+        for r in range(world):
+            assert np.abs(results[r] - ref).max() <= bound
+            np.testing.assert_array_equal(results[r], results[0])
+        assert np.all(results[0][1] == 0)
 
 
 def test_shard_ranges_cover_the_cache_once():

@@ -284,8 +284,10 @@ def test_context_parallel_shards(cuda_device, oracle_lib):
     """E4M3 cache split by slot range over 3 emulated ranks: records stacked and combined."""
     from test_parity_gpu import _shards_combined
     w = _random_case(2800, 200, 16, 2, 16384, 2051, minus1=0.05, widths=True)
-    got, _ = _shards_combined(w, dev(w, cuda_device), 3, k_scale=w.k_scale, v_scale=w.v_scale)
-    compare(w, got, oracle_lib, 1.0 / 16.0, None, "e4m3 context parallel R=3")
+    for rec in (torch.float32, torch.bfloat16):
+        got, _ = _shards_combined(w, dev(w, cuda_device), 3, k_scale=w.k_scale,
+                                  v_scale=w.v_scale, record_dtype=rec)
+        compare(w, got, oracle_lib, 1.0 / 16.0, None, f"e4m3 context parallel R=3 {rec}")
 
 
 def test_cache_offsets_beyond_4gib(cuda_device, oracle_lib):

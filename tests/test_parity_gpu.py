@@ -651,13 +651,14 @@ def _shards_combined(w, d, R, scale=1.0 / 16.0, nsplit=0, **kw):
     return out.cpu(), rec_l
 
 
+@pytest.mark.parametrize("rec", [torch.float32, torch.bfloat16], ids=["fp32", "bf16"])
 @pytest.mark.parametrize("R", [1, 2, 3, 5])
-def test_context_parallel_shards(cuda_device, oracle_lib, R):
+def test_context_parallel_shards(cuda_device, oracle_lib, R, rec):
     w = _random_case(90 + R, 300, 16, 2, 16384, 2051, minus1=0.05, widths=True)
     d = dev(w, cuda_device)
-    got, rec_l = _shards_combined(w, d, R)
+    got, rec_l = _shards_combined(w, d, R, record_dtype=rec)
     ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0)
-    check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"context parallel R={R}")
+    check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"context parallel R={R} {rec}")
     if R == 1:  # one shard holding the whole cache: bitwise the unsharded call
         assert torch.equal(got.view(torch.int16), run(d, 1.0 / 16.0).view(torch.int16))
     for t in empty_rows(w):
@@ -668,15 +669,19 @@ def test_context_parallel_wide_rows_and_decode(cuda_device, oracle_lib):
     """W = 6,000 (each shard combines its own splits into one record) and a decode-shape
     batch with forced split counts."""
     w = _random_case(95, 120, 16, 2, 20000, 6000, minus1=0.1, widths=True)
-    got, _ = _shards_combined(w, dev(w, cuda_device), 3)
     rows = list(range(0, w.Tq, 4))
     ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, w.width, 1.0 / 16.0, rows=rows)
-    check_gates(got[rows].float(), torch.from_numpy(ref), empty_rows(w, rows), "context parallel W=6000")
+    for rec in (torch.float32, torch.bfloat16):  # the shards' own splits combine into bf16 too
+        got, _ = _shards_combined(w, dev(w, cuda_device), 3, record_dtype=rec)
+        check_gates(got[rows].float(), torch.from_numpy(ref), empty_rows(w, rows),
+                    f"context parallel W=6000 {rec}")
     w = _random_case(96, 3, 16, 2, 65536, 2051, minus1=0.2)
+    ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
     for nsplit in (1, 4, 16):
-        got, _ = _shards_combined(w, dev(w, cuda_device), 2, nsplit=nsplit)
-        ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0)
-        check_gates(got.float(), torch.from_numpy(ref), empty_rows(w), f"context parallel decode n={nsplit}")
+        for rec in (torch.float32, torch.bfloat16):
+            got, _ = _shards_combined(w, dev(w, cuda_device), 2, nsplit=nsplit, record_dtype=rec)
+            check_gates(got.float(), torch.from_numpy(ref), empty_rows(w),
+                        f"context parallel decode n={nsplit} {rec}")
 
 
 def test_context_parallel_block4_and_empty_shard(cuda_device, oracle_lib):
@@ -685,13 +690,13 @@ def test_context_parallel_block4_and_empty_shard(cuda_device, oracle_lib):
     w = _random_case(97, 64, 16, 2, 4096, 300, minus1=0.1)
     w.slot_idx = wl.uniform_distinct(torch.Generator().manual_seed(98), 64, 1024, 300)
     w.block = 4
-    got, _ = _shards_combined(w, dev(w, cuda_device), 3)
+    got, _ = _shards_combined(w, dev(w, cuda_device), 3, record_dtype=torch.bfloat16)
     ref = oracle_lib.forward(w.q, w.k_cache, w.v_cache, w.slot_idx, None, 1.0 / 16.0, block=4)
     check_gates(got.float(), torch.from_numpy(ref), None, "context parallel block4")
     t = _random_case(99, 8, 16, 2, 12, 10, minus1=0.0)
     t.block = 4  # 3 blocks over 4 ranks
     t.slot_idx = torch.tensor([[0, 1, 2, -1, -1, -1, -1, -1, -1, -1]] * 8, dtype=torch.int32)
-    got, rec_l = _shards_combined(t, dev(t, cuda_device), 4)
+    got, rec_l = _shards_combined(t, dev(t, cuda_device), 4, record_dtype=torch.bfloat16)
     assert torch.isinf(rec_l[3]).all()
     ref = oracle_lib.forward(t.q, t.k_cache, t.v_cache, t.slot_idx, None, 1.0 / 16.0, block=4)
     check_gates(got.float(), torch.from_numpy(ref), None, "context parallel empty shard")

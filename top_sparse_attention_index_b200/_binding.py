@@ -45,9 +45,9 @@ SIGNATURES = {
                                         _p, _i64, _i64, _i32, _p, _sz, _p, _p]),
     "qsa_sparse_prefill_partial": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _i32,
-                                          _i64, _i64, _i32, _f, _f, _f, _p, _p, _i32, _p, _sz, _p,
-                                          _p]),
-    "qsa_combine_partials": (_i32, [_p, _p, _i32, _i32, _i32, _i32, _p, _i64, _i64, _p]),
+                                          _i64, _i64, _i32, _f, _f, _f, _p, _p, _i32, _i32, _p,
+                                          _sz, _p, _p]),
+    "qsa_combine_partials": (_i32, [_p, _p, _i32, _i32, _i32, _i32, _i32, _p, _i64, _i64, _p]),
     "qsa_sparse_prefill_noalloc": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _f, _p,
                                           _i64, _i64, _i32, _p, _p]),
@@ -176,21 +176,21 @@ def qsa_sparse_prefill_fp8kv(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_s
 def qsa_sparse_prefill_partial(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
                                v_cache, v_stride_s, v_stride_h, slot_idx, idx_stride_t, width, Tq,
                                Hq, Hkv, D, S, W, block, slot_lo, S_total, kv_fp8, scale, k_scale,
-                               v_scale, part_o, part_lse, nsplit, workspace, workspace_bytes,
-                               err_word, stream) -> int:
+                               v_scale, part_o, part_lse, record_bf16, nsplit, workspace,
+                               workspace_bytes, err_word, stream) -> int:
     """Raw call of one slot-range shard's partial record (context parallelism)."""
     return int(load_library().qsa_sparse_prefill_partial(
         q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache, v_stride_s,
         v_stride_h, slot_idx, idx_stride_t, width, Tq, Hq, Hkv, D, S, W, block, slot_lo, S_total,
         kv_fp8, ctypes.c_float(scale), ctypes.c_float(k_scale), ctypes.c_float(v_scale), part_o,
-        part_lse, nsplit, workspace, workspace_bytes, err_word, stream))
+        part_lse, record_bf16, nsplit, workspace, workspace_bytes, err_word, stream))
 
 
-def qsa_combine_partials(part_o, part_lse, R, Tq, Hq, D, out, out_stride_t, out_stride_h,
-                         stream) -> int:
+def qsa_combine_partials(part_o, part_lse, record_bf16, R, Tq, Hq, D, out, out_stride_t,
+                         out_stride_h, stream) -> int:
     """Raw call of the log-sum-exp combine of R stacked partial records."""
-    return int(load_library().qsa_combine_partials(part_o, part_lse, R, Tq, Hq, D, out,
-                                                   out_stride_t, out_stride_h, stream))
+    return int(load_library().qsa_combine_partials(part_o, part_lse, record_bf16, R, Tq, Hq, D,
+                                                   out, out_stride_t, out_stride_h, stream))
 
 
 def qsa_sparse_prefill_noalloc(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h,
@@ -281,15 +281,16 @@ def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=No
 
 def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, width=None,
                            scale=None, part_o=None, part_lse=None, nsplit=0, err_word=None,
-                           stream=None, block=1, k_scale=1.0, v_scale=1.0):
+                           stream=None, block=1, k_scale=1.0, v_scale=1.0,
+                           record_dtype=torch.float32):
     """One device's partial record for a cache split by slot range (context parallel).
 
     k_cache / v_cache hold the global slots [slot_lo, slot_lo + S) of a cache of S_total
     slots (bf16, or float8_e4m3fn codes with k_scale / v_scale); slot_idx holds global
-    slot numbers.  Returns (part_o fp32 [Tq, Hq, 256], part_lse fp32 [Tq, Hq]): the output
-    normalised over this device's valid slots and the base-2 log-sum-exp of their scaled
-    scores (-inf where there are none).  Combine the records of all devices with
-    combine_partials.
+    slot numbers.  Returns (part_o [Tq, Hq, 256] of record_dtype (float32 or bfloat16),
+    part_lse fp32 [Tq, Hq]): the output normalised over this device's valid slots and the
+    base-2 log-sum-exp of their scaled scores (-inf where there are none).  Combine the
+    records of all devices with combine_partials.
     """
     device = q.device
     if device.type != "cuda":
@@ -308,13 +309,16 @@ def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, widt
         _check_dev(name, t, dt, device)
     if width is not None:
         _check_dev("width", width, torch.int32, device)
+    if record_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("record_dtype must be torch.float32 or torch.bfloat16")
     if part_o is None:
-        part_o = torch.empty(Tq, Hq, D, dtype=torch.float32, device=device)
+        part_o = torch.empty(Tq, Hq, D, dtype=record_dtype, device=device)
     if part_lse is None:
         part_lse = torch.empty(Tq, Hq, dtype=torch.float32, device=device)
-    for name, t, shape in (("part_o", part_o, (Tq, Hq, D)), ("part_lse", part_lse, (Tq, Hq))):
-        if tuple(t.shape) != shape or t.dtype != torch.float32 or not t.is_contiguous() or t.device != device:
-            raise ValueError(f"{name} must be a contiguous float32 {shape} tensor on {device}")
+    for name, t, shape, dt in (("part_o", part_o, (Tq, Hq, D), record_dtype),
+                               ("part_lse", part_lse, (Tq, Hq), torch.float32)):
+        if tuple(t.shape) != shape or t.dtype != dt or not t.is_contiguous() or t.device != device:
+            raise ValueError(f"{name} must be a contiguous {dt} {shape} tensor on {device}")
     if scale is None:
         scale = 1.0 / (D ** 0.5)
     if stream is None:
@@ -328,8 +332,8 @@ def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, widt
             _ptr(v_cache), v_cache.stride(0), v_cache.stride(1), _ptr(slot_idx) if W else None,
             slot_idx.stride(0), _ptr(width), Tq, Hq, Hkv, D, S, W, block, int(slot_lo),
             int(S_total), 1 if kv_fp8 else 0, float(scale), float(k_scale), float(v_scale),
-            _ptr(part_o), _ptr(part_lse), ns, _ptr(ws), ws_bytes, _ptr(err_word),
-            stream.cuda_stream)
+            _ptr(part_o), _ptr(part_lse), 1 if record_dtype == torch.bfloat16 else 0, ns,
+            _ptr(ws), ws_bytes, _ptr(err_word), stream.cuda_stream)
     if st != QSA_OK:
         raise QSAError(st, qsa_last_error_detail())
     return part_o, part_lse
@@ -337,16 +341,20 @@ def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, widt
 
 def combine_partials(part_o, part_lse, out=None, stream=None):
     """bf16 [Tq, Hq, 256]: the log-sum-exp combine of R stacked partial records
-    (part_o fp32 [R, Tq, Hq, 256], part_lse fp32 [R, Tq, Hq], both contiguous)."""
+    (part_o float32 or bfloat16 [R, Tq, Hq, 256], part_lse float32 [R, Tq, Hq], both
+    contiguous)."""
     device = part_o.device
     if device.type != "cuda":
         raise ValueError("combine_partials runs on CUDA tensors only")
     if part_o.dim() != 4 or part_lse.shape != part_o.shape[:3]:
         raise ValueError("part_o must be [R, Tq, Hq, D] and part_lse [R, Tq, Hq]")
     R, Tq, Hq, D = part_o.shape
+    if part_o.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("part_o must be float32 or bfloat16")
     for name, t in (("part_o", part_o), ("part_lse", part_lse)):
-        if t.dtype != torch.float32 or not t.is_contiguous() or t.device != device:
-            raise ValueError(f"{name} must be a contiguous float32 tensor on {device}")
+        dt = part_o.dtype if name == "part_o" else torch.float32
+        if t.dtype != dt or not t.is_contiguous() or t.device != device:
+            raise ValueError(f"{name} must be a contiguous {dt} tensor on {device}")
     if out is None:
         out = torch.empty(Tq, Hq, D, dtype=torch.bfloat16, device=device)
     else:
@@ -354,8 +362,9 @@ def combine_partials(part_o, part_lse, out=None, stream=None):
     if stream is None:
         stream = torch.cuda.current_stream(device)
     with torch.cuda.device(device):
-        st = qsa_combine_partials(_ptr(part_o), _ptr(part_lse), R, Tq, Hq, D, _ptr(out),
-                                  out.stride(0), out.stride(1), stream.cuda_stream)
+        st = qsa_combine_partials(_ptr(part_o), _ptr(part_lse),
+                                  1 if part_o.dtype == torch.bfloat16 else 0, R, Tq, Hq, D,
+                                  _ptr(out), out.stride(0), out.stride(1), stream.cuda_stream)
     if st != QSA_OK:
         raise QSAError(st, qsa_last_error_detail())
     return out

@@ -5,9 +5,11 @@ group (decode context parallelism, named for this attention path in the article
 
 Every rank holds a contiguous slot range of the cache and sees the same global selection.
 Each rank computes its partial record in the CUDA kernels (qsa_sparse_prefill_partial:
-the output normalised over its own slots and their base-2 log-sum-exp); the records are
-exchanged with one all-gather (torch.distributed, NCCL on GPUs) and combined in the CUDA
-combine kernel (qsa_combine_partials), which gives the attention over the whole cache.
+the output normalised over its own slots, bf16 by default, and the fp32 base-2
+log-sum-exp of their scores); the records are exchanged with one all-gather
+(torch.distributed, NCCL on GPUs) and combined in the CUDA combine kernel
+(qsa_combine_partials), which gives the attention over the whole cache.  bf16 records
+halve the bytes every rank sends (512 instead of 1,024 per (query row, head)).
 This module only shards, exchanges and marshals: the arithmetic is in the kernels.
 """
 from __future__ import annotations
@@ -53,11 +55,13 @@ def exchange_records(part_o: torch.Tensor, part_lse: torch.Tensor, group=None):
 
 def sparse_prefill_context_parallel(q, k_local, v_local, slot_idx, slot_lo, S_total,
                                     group=None, width=None, scale=None, block=1, k_scale=1.0,
-                                    v_scale=1.0, out=None, partial_fn=None, combine_fn=None):
+                                    v_scale=1.0, out=None, partial_fn=None, combine_fn=None,
+                                    record_dtype=torch.bfloat16):
     """Selected-slot sparse attention over a cache split by slot range across the ranks of
     `group`: this rank's k_local / v_local hold global slots [slot_lo, slot_lo + S_local)
     (see shard_ranges); q, slot_idx (global slot numbers) and width are the same on every
-    rank.  Returns the bf16 output [Tq, Hq, 256] on every rank.
+    rank.  Returns the bf16 output [Tq, Hq, 256] on every rank.  record_dtype (bfloat16 or
+    float32) is the type of the exchanged normalised outputs.
 
     partial_fn / combine_fn default to the CUDA entry points (sparse_prefill_partial,
     combine_partials); they are parameters so that the exchange can be exercised on hosts
@@ -66,6 +70,7 @@ def sparse_prefill_context_parallel(q, k_local, v_local, slot_idx, slot_lo, S_to
     partial_fn = partial_fn or _binding.sparse_prefill_partial
     combine_fn = combine_fn or _binding.combine_partials
     part_o, part_lse = partial_fn(q, k_local, v_local, slot_idx, slot_lo, S_total, width=width,
-                                  scale=scale, block=block, k_scale=k_scale, v_scale=v_scale)
+                                  scale=scale, block=block, k_scale=k_scale, v_scale=v_scale,
+                                  record_dtype=record_dtype)
     g_o, g_l = exchange_records(part_o, part_lse, group)
     return combine_fn(g_o, g_l, out=out)

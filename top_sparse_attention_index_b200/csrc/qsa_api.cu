@@ -149,7 +149,7 @@ uint64_t current_context_id() {
 
 extern "C" {
 
-int32_t qsa_abi_version(void) { return 1; }
+int32_t qsa_abi_version(void) { return 2; }
 
 const char* qsa_status_string(qsa_status_t status) {
   switch (status) {
@@ -198,8 +198,9 @@ namespace {
 struct PartialArgs {
   int64_t slot_lo = 0;
   int64_t S_total = -1;  // -1: S (unsharded)
-  float* part_o = nullptr;
-  float* part_lse = nullptr;  // both set: write one normalised fp32 record + base-2 LSE
+  void* part_o = nullptr;
+  float* part_lse = nullptr;  // both set: write one normalised record + base-2 LSE
+  bool rec_bf16 = false;      // the record's O in bf16 (else fp32)
 };
 
 // The body shared by every launching entry point.  kv_fp8: k_cache / v_cache hold E4M3
@@ -339,8 +340,9 @@ qsa_status_t prefill_impl(const void* q, int64_t q_stride_t, int64_t q_stride_h,
     p.partial_out = 1;
     p.part_o = part.part_o;
     p.part_lse = part.part_lse;
+    p.rec_bf16 = part.rec_bf16 ? 1 : 0;
     if (pl.nsplit == 1) {  // the single split's record is the partial record itself
-      p.ws_o = part.part_o;
+      p.ws_o = part.rec_bf16 ? nullptr : static_cast<float*>(part.part_o);
       p.ws_lse = part.part_lse;
     }
   }
@@ -377,15 +379,19 @@ qsa_status_t qsa_sparse_prefill_partial(const void* q, int64_t q_stride_t, int64
                                         const int32_t* width, int32_t Tq, int32_t Hq, int32_t Hkv,
                                         int32_t D, int64_t S, int32_t W, int32_t block,
                                         int64_t slot_lo, int64_t S_total, int32_t kv_fp8,
-                                        float scale, float k_scale, float v_scale, float* part_o,
-                                        float* part_lse, int32_t nsplit, void* workspace,
-                                        size_t workspace_bytes, uint32_t* err_word, void* stream) {
+                                        float scale, float k_scale, float v_scale, void* part_o,
+                                        float* part_lse, int32_t record_bf16, int32_t nsplit,
+                                        void* workspace, size_t workspace_bytes,
+                                        uint32_t* err_word, void* stream) {
   if (kv_fp8 != 0 && kv_fp8 != 1) return fail(QSA_ERR_INVALID_ARG, "kv_fp8 must be 0 or 1");
+  if (record_bf16 != 0 && record_bf16 != 1)
+    return fail(QSA_ERR_INVALID_ARG, "record_bf16 must be 0 or 1");
   PartialArgs part;
   part.slot_lo = slot_lo;
   part.S_total = S_total;
   part.part_o = part_o;
   part.part_lse = part_lse;
+  part.rec_bf16 = record_bf16 != 0;
   if (Tq > 0 && (part_o == nullptr || part_lse == nullptr)) {
     g_detail[0] = '\0';
     return fail(QSA_ERR_INVALID_ARG, "NULL part_o or part_lse");
@@ -397,10 +403,12 @@ qsa_status_t qsa_sparse_prefill_partial(const void* q, int64_t q_stride_t, int64
                       nullptr, 0, 0, nsplit, workspace, workspace_bytes, err_word, stream, part);
 }
 
-qsa_status_t qsa_combine_partials(const float* part_o, const float* part_lse, int32_t R,
-                                  int32_t Tq, int32_t Hq, int32_t D, void* out,
+qsa_status_t qsa_combine_partials(const void* part_o, const float* part_lse, int32_t record_bf16,
+                                  int32_t R, int32_t Tq, int32_t Hq, int32_t D, void* out,
                                   int64_t out_stride_t, int64_t out_stride_h, void* stream) {
   g_detail[0] = '\0';
+  if (record_bf16 != 0 && record_bf16 != 1)
+    return fail(QSA_ERR_INVALID_ARG, "record_bf16 must be 0 or 1");
   if (R < 1 || Tq < 0 || Hq < 1)
     return fail(QSA_ERR_INVALID_ARG, "bad sizes: R=%d Tq=%d Hq=%d", R, Tq, Hq);
   if (D != qsa::kHeadDim) return fail(QSA_ERR_UNSUPPORTED, "head dimension %d (only 256)", D);
@@ -414,8 +422,9 @@ qsa_status_t qsa_combine_partials(const float* part_o, const float* part_lse, in
   if (int64_t(Tq) * Hq > int64_t(INT32_MAX) * 4)
     return fail(QSA_ERR_INVALID_ARG, "too many rows for one launch");
   qsa::FwdParams p{};
-  p.ws_o = const_cast<float*>(part_o);
+  p.ws_o = static_cast<float*>(const_cast<void*>(part_o));
   p.ws_lse = const_cast<float*>(part_lse);
+  p.in_bf16 = record_bf16;
   p.out = static_cast<uint16_t*>(out);
   p.out_stride_t = out_stride_t;
   p.out_stride_h = out_stride_h;

@@ -278,10 +278,19 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
       for (int g = tid; g < G; g += C::kThreads)
         p.ws_lse[(int64_t(split) * p.Tq + t) * p.Hq + head0 + g] = kNegInf;
       if (p.nsplit == 1) {  // a partial record (the combine skips it): O written as zeros
-        for (int i = tid; i < G * (kHeadDim / 4); i += C::kThreads) {
-          const int g = i / (kHeadDim / 4), c = i % (kHeadDim / 4);
-          reinterpret_cast<float4*>(p.ws_o + (int64_t(t) * p.Hq + head0 + g) * kHeadDim)[c] =
-              make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p.rec_bf16) {
+          for (int i = tid; i < G * kChunks; i += C::kThreads) {
+            const int g = i / kChunks, c = i % kChunks;
+            reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.part_o) +
+                                     (int64_t(t) * p.Hq + head0 + g) * kHeadDim)[c] =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+        } else {
+          for (int i = tid; i < G * (kHeadDim / 4); i += C::kThreads) {
+            const int g = i / (kHeadDim / 4), c = i % (kHeadDim / 4);
+            reinterpret_cast<float4*>(p.ws_o + (int64_t(t) * p.Hq + head0 + g) * kHeadDim)[c] =
+                make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
       }
     }
@@ -794,9 +803,18 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
       *reinterpret_cast<uint4*>(p.out + int64_t(t) * p.out_stride_t + h * p.out_stride_h + dg * 8) = v;
     } else {
       const int64_t row = (int64_t(split) * p.Tq + t) * p.Hq + h;
-      float4* dst = reinterpret_cast<float4*>(p.ws_o + row * kHeadDim + dg * 8);
-      dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-      dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+      if (p.nsplit == 1 && p.rec_bf16) {  // the record itself, O in bf16 (RNE)
+        uint4 v;
+        v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+        v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+        *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.part_o) + row * kHeadDim + dg * 8) = v;
+      } else {
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + row * kHeadDim + dg * 8);
+        dst[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        dst[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+      }
       if (dg == 0) p.ws_lse[row] = mstar + fast_log2(lsum);
     }
   }
@@ -808,6 +826,9 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
 // its eight elements of D, with the partial rows read regardless of their weight (the
 // buffers hold every split's row) so that the reads of several splits are in flight at
 // once; a split with lse = -inf (empty, its row never written) is left out by a select.
+// IN_BF16: the partial rows are bf16 (gathered context-parallel records), else fp32.
+// With partial_out the result is one record (O fp32, or bf16 with rec_bf16, and its LSE).
+template <bool IN_BF16>
 __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p) {
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   const int64_t row = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
@@ -819,15 +840,27 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, off));
   const int64_t t = row / p.Hq, h = row % p.Hq;
-  if (mstar == kNegInf) {  // no valid slot in any split
-    if (p.partial_out) {
-      float4* po = reinterpret_cast<float4*>(p.part_o + row * kHeadDim + lane * 8);
-      po[0] = po[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (lane == 0) p.part_lse[row] = kNegInf;
+  // writes eight elements of this lane: a record (fp32 or bf16) or the bf16 output
+  auto store8 = [&](const float (&x)[8]) {
+    uint4 v;
+    v.x = pack_bf16x2(x[0], x[1]);
+    v.y = pack_bf16x2(x[2], x[3]);
+    v.z = pack_bf16x2(x[4], x[5]);
+    v.w = pack_bf16x2(x[6], x[7]);
+    if (p.partial_out && !p.rec_bf16) {
+      float4* po = reinterpret_cast<float4*>(static_cast<float*>(p.part_o) + row * kHeadDim + lane * 8);
+      po[0] = make_float4(x[0], x[1], x[2], x[3]);
+      po[1] = make_float4(x[4], x[5], x[6], x[7]);
+    } else if (p.partial_out) {
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.part_o) + row * kHeadDim + lane * 8) = v;
     } else {
-      *reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8) =
-          make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8) = v;
     }
+  };
+  if (mstar == kNegInf) {  // no valid slot in any split
+    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    store8(z);
+    if (p.partial_out && lane == 0) p.part_lse[row] = kNegInf;
     return;
   }
   float acc[8];
@@ -840,31 +873,35 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
 #pragma unroll 4
     for (int i = 0; i < cnt; ++i) {
       const float lse = __shfl_sync(0xffffffffu, lse_l, i);
-      const float4* src =
-          reinterpret_cast<const float4*>(p.ws_o + ((s0 + i) * rows + row) * kHeadDim + lane * 8);
-      const float4 a = src[0], b = src[1];
+      const int64_t off = ((s0 + i) * rows + row) * kHeadDim + lane * 8;
+      float x[8];
+      if constexpr (IN_BF16) {
+        const uint4 r = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(p.ws_o) + off);
+        x[0] = bf16lo_to_f32(r.x); x[1] = bf16hi_to_f32(r.x);
+        x[2] = bf16lo_to_f32(r.y); x[3] = bf16hi_to_f32(r.y);
+        x[4] = bf16lo_to_f32(r.z); x[5] = bf16hi_to_f32(r.z);
+        x[6] = bf16lo_to_f32(r.w); x[7] = bf16hi_to_f32(r.w);
+      } else {
+        const float4 a = reinterpret_cast<const float4*>(p.ws_o + off)[0];
+        const float4 b = reinterpret_cast<const float4*>(p.ws_o + off)[1];
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+      }
       if (lse != kNegInf) {  // warp-uniform
         const float w = fast_exp2(lse - mstar);
         wsum += w;
-        acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
-        acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += w * x[e];
       }
     }
   }
   const float inv = 1.f / wsum;
-  if (p.partial_out) {  // one normalised record of all splits: O and lse* + log2(sum of weights)
-    float4* po = reinterpret_cast<float4*>(p.part_o + row * kHeadDim + lane * 8);
-    po[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    po[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-    if (lane == 0) p.part_lse[row] = mstar + fast_log2(wsum);
-    return;
-  }
-  uint4 v;
-  v.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  v.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  v.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-  v.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  *reinterpret_cast<uint4*>(p.out + t * p.out_stride_t + h * p.out_stride_h + lane * 8) = v;
+  float res[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) res[e] = acc[e] * inv;
+  store8(res);
+  // one normalised record of all splits: O and lse* + log2(sum of weights)
+  if (p.partial_out && lane == 0) p.part_lse[row] = mstar + fast_log2(wsum);
 }
 
 template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8,
@@ -1125,7 +1162,10 @@ cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream) {
   const int64_t rows = int64_t(p.Tq) * p.Hq;
   if (rows == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
-  qsa_lse_combine_kernel<<<grid, 128, 0, stream>>>(p);
+  if (p.in_bf16)
+    qsa_lse_combine_kernel<true><<<grid, 128, 0, stream>>>(p);
+  else
+    qsa_lse_combine_kernel<false><<<grid, 128, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

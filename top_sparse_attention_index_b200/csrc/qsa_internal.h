@@ -58,8 +58,10 @@ struct FwdParams {
   // 1: write the normalised fp32 O and the base-2 LSE (ws_o / ws_lse layout, the call's
   // own split plan combined into one record per (t, h)) instead of bf16 out
   int32_t partial_out;
-  float* part_o;            // partial_out: fp32 [Tq, Hq, D]
+  void* part_o;             // partial_out: [Tq, Hq, D], fp32 or bf16 (rec_bf16)
   float* part_lse;          // partial_out: fp32 [Tq, Hq]
+  int32_t rec_bf16;         // partial_out: the record's O is bf16 (else fp32)
+  int32_t in_bf16;          // combine of gathered records: ws_o holds bf16 O (else fp32)
 };
 
 // Kernel configuration chosen for a group size G (shared by planner and launcher).

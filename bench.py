@@ -33,6 +33,7 @@ ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
 from top_sparse_attention_index_b200 import workloads as wl  # noqa: E402
+from top_sparse_attention_index_b200.gather_probe import PROBE_CONFIGS, gather_peak  # noqa: E402,F401
 
 METRIC = "sparse prefill TFLOP/s & query-slot pairs/s, 7810q×2051 sel; % of roofline"
 
@@ -375,7 +376,7 @@ def main():
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # the SM-side roofline, measured right after the timed region on the same device
-    probe = gather_peak(device, 256 if w.kv_format == "e4m3" else 512)
+    probe = gather_peak(device, 256 if w.kv_format == "e4m3" else 512)  # (gather_probe.py)
 
     if dist is not None:
         dist.destroy_process_group()
@@ -442,64 +443,6 @@ def main():
     if not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(result))
-
-
-# The gather probe (include/qsa_probe.h) measures, live on the device, the rate at which
-# the SMs pull random rows of an L2-resident 64 MB buffer into shared memory and read each
-# landed row back once with ldmatrix -- the data movement of the fused kernel without its
-# arithmetic -- with the fused kernel's own loader (cp.async, method 0) and with TMA
-# tile::gather4 (method 1), over a few pipeline shapes (warps per CTA, stages, CTAs per
-# SM).  The best rate is the SM-side roofline of a launch whose gathered rows are L2 hits.
-PROBE_BUFFER_BYTES = 64 << 20
-PROBE_CONFIGS = {
-    512: [(12, 2, 1), (8, 3, 1), (6, 2, 2), (2, 4, 3)],
-    256: [(15, 3, 1), (12, 4, 1), (4, 4, 3), (6, 4, 2)],
-}
-
-
-def gather_peak(device, row_bytes: int, reps: int = 5) -> dict:
-    """Best gather rate (TB/s) of the probe over its methods and pipeline shapes."""
-    import top_sparse_attention_index_b200 as qsa
-    sms = torch.cuda.get_device_properties(device).multi_processor_count
-    gen = torch.Generator(device=device).manual_seed(99)
-    buf = torch.randint(-2**31, 2**31 - 1, (PROBE_BUFFER_BYTES // 4,), dtype=torch.int32,
-                        device=device, generator=gen)
-    sink = torch.zeros(258, dtype=torch.int32, device=device)
-    stream = torch.cuda.current_stream(device)
-    rows = PROBE_BUFFER_BYTES // row_bytes
-    runs = []
-    for method in (0, 1):
-        for warps, stages, per_sm in PROBE_CONFIGS[row_bytes]:
-            ctas = sms * per_sm
-            iters = max(4, int(2e9 / (ctas * warps * 16 * row_bytes)))
-            moved = ctas * warps * iters * 16 * row_bytes
-            sink.zero_()
-
-            def launch(seed):
-                st = qsa.qsa_probe_gather(method, 1, buf.data_ptr(), rows, row_bytes, row_bytes,
-                                          warps, stages, ctas, iters, seed, sink.data_ptr(),
-                                          stream.cuda_stream)
-                if st != qsa.QSA_OK:
-                    raise qsa.QSAError(st, qsa.qsa_last_error_detail())
-
-            launch(1)
-            launch(2)
-            times = []
-            for r in range(reps):
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                launch(3 + r)
-                b.record(stream)
-                torch.cuda.synchronize(device)
-                times.append(a.elapsed_time(b) * 1e-3)
-            ok = int(sink[0].item()) == 0
-            runs.append({"method": ["cp.async", "tma gather4"][method], "warps_per_cta": warps,
-                         "stages": stages, "ctas_per_sm": per_sm,
-                         "tb_per_s": moved / statistics.median(times) / 1e12 if ok else None})
-    best = max((r for r in runs if r["tb_per_s"] is not None), key=lambda r: r["tb_per_s"])
-    return {"tb_per_s": best["tb_per_s"], "best": best, "runs": runs, "row_bytes": row_bytes,
-            "buffer_bytes": PROBE_BUFFER_BYTES, "read_back": True}
 
 
 def _code_only(text: str) -> str:

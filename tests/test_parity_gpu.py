@@ -648,6 +648,7 @@ def _shards_combined(w, d, R, scale=1.0 / 16.0, nsplit=0, **kw):
         rec_l.append(pl)
     out = qsa.combine_partials(torch.stack(rec_o), torch.stack(rec_l))
     torch.cuda.synchronize()
+    _shards_combined.last_records = rec_o
     return out.cpu(), rec_l
 
 
@@ -663,6 +664,8 @@ def test_context_parallel_shards(cuda_device, oracle_lib, R, rec):
         assert torch.equal(got.view(torch.int16), run(d, 1.0 / 16.0).view(torch.int16))
     for t in empty_rows(w):
         assert all(torch.isinf(l[t]).all() for l in rec_l)
+        # a record with no valid slot holds zeros (the documented record content)
+        assert all((o[t] == 0).all() for o in _shards_combined.last_records)
 
 
 def test_context_parallel_wide_rows_and_decode(cuda_device, oracle_lib):

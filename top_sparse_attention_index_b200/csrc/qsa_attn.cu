@@ -278,20 +278,12 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
       for (int g = tid; g < G; g += C::kThreads)
         p.ws_lse[(int64_t(split) * p.Tq + t) * p.Hq + head0 + g] = kNegInf;
       if (p.nsplit == 1) {  // a partial record (the combine skips it): O written as zeros
-        if (p.rec_bf16) {
-          for (int i = tid; i < G * kChunks; i += C::kThreads) {
-            const int g = i / kChunks, c = i % kChunks;
-            reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.part_o) +
-                                     (int64_t(t) * p.Hq + head0 + g) * kHeadDim)[c] =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-        } else {
-          for (int i = tid; i < G * (kHeadDim / 4); i += C::kThreads) {
-            const int g = i / (kHeadDim / 4), c = i % (kHeadDim / 4);
-            reinterpret_cast<float4*>(p.ws_o + (int64_t(t) * p.Hq + head0 + g) * kHeadDim)[c] =
-                make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
+        // (the group's G rows are contiguous; 2- or 4-byte elements)
+        const int64_t esz = p.rec_bf16 ? 2 : 4;
+        uint4* z = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.part_o) +
+                                            (int64_t(t) * p.Hq + head0) * kHeadDim * esz);
+        const int n16 = int(G * kHeadDim * esz / 16);
+        for (int i = tid; i < n16; i += C::kThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     return;

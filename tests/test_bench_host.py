@@ -102,3 +102,20 @@ def test_gather_probe_shapes_fit_one_sm():
             smem = warps * stages * 16 * row_bytes + 2 * warps * stages * 8
             assert smem <= 227 * 1024
             assert per_sm * (smem + 1024) <= 228 * 1024
+
+def test_binding_roofline_is_the_slower_bound():
+    """The long prefill's rows are L2 hits: the gather bound (algorithmic bytes against the
+    gather probe) binds.  A cache twice the size of L2 moves most rows from DRAM: the
+    DRAM bound (measured traffic against the copy bandwidth) binds.  Without a traffic
+    record of the current kernel only the gather bound is known."""
+    probe = {"tb_per_s": 18.0, "runs": [{}] * 8, "best": {}}
+    lp = bench._rooflines(33e9 / 2.02e-3 / 1e9, 33e9, 2.02e-3, probe, 1.76e9, None, 6548.8, "m")
+    assert lp["roofline"]["bound"] == "l2" and lp["roofline"] is lp["l2_gather"]
+    assert abs(lp["roofline"]["frac"] - (33e9 / 2.02e-3) / 18e12) < 1e-9
+    assert abs(lp["hbm"]["frac"] - 1.76e9 / 2.02e-3 / 6548.8e9) < 1e-9
+    mx = bench._rooflines(8.65e9 / 0.922e-3 / 1e9, 8.65e9, 0.922e-3, probe, 5.9e9, None,
+                          6548.8, "m")
+    assert mx["roofline"]["bound"] == "hbm" and mx["roofline"] is mx["hbm"]
+    assert abs(mx["roofline"]["frac"] - 5.9e9 / 0.922e-3 / 6548.8e9) < 1e-9
+    none = bench._rooflines(1.0, 8.65e9, 0.922e-3, probe, None, None, 6548.8, "m")
+    assert none["roofline"]["bound"] == "l2" and none["hbm"]["frac"] is None

@@ -138,8 +138,9 @@ template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool
           int QROWS, bool TMA>
 __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     qsa_sparse_attn_fwd_kernel(const FwdParams p, const __grid_constant__ TmaMaps maps) {
-  static_assert(!QSPLIT || DSPLIT == 2, "splitting Q K^T needs a D-split pair");
-  constexpr int kKS = QSPLIT ? 8 : 16;  // k-steps of Q K^T per warp
+  static_assert(!QSPLIT || DSPLIT == 2 || (DSPLIT == 4 && !KV8),
+                "splitting Q K^T needs a D-split pair (or a bf16 D-split quad)");
+  constexpr int kKS = QSPLIT ? 16 / DSPLIT : 16;  // k-steps of Q K^T per warp
   using C = Cfg<NTILE, DSPLIT, SL, STAGES, KV8, SLOT16, QROWS, TMA>;
   using SlotT = std::conditional_t<SLOT16, uint16_t, uint32_t>;
   constexpr int kKvRow = C::kKvRow;
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
   // Gather addressing: global-space row bases, a row = base + slot * stride in bytes (one
   // 32x32->64-bit mad per row and tensor in the loop) and, per lane, the eight swizzled
   // chunk offsets (row & 7 is a compile-time
-  // constant in the unrolled loop because a lane's rows start at 0 or 8), so a
+  // constant in the unrolled loop up to the warp's first row, 0, 4 or 8), so a
   // destination is a register plus an immediate.
   // An E4M3 row is 16 chunks: lanes 0-15 copy one row, lanes 16-31 the next.
   constexpr int kElem = KV8 ? 1 : 2;
@@ -358,7 +359,8 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     } else if constexpr (!KV8) {
       uint32_t kd[8];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (m << 4));
+      for (int m = 0; m < 8; ++m)  // (row0 & 7 is 0 for a pair's warps, 0 or 4 for a quad's)
+        kd[m] = sub_rows + buf * C::kSubBytes + (lane16 ^ (uint32_t((m + row0) & 7) << 4));
 #pragma unroll
       for (int i = 0; i < kLoadRows; i += 4) {
         uint32_t sl[4];
@@ -576,7 +578,7 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
 #pragma unroll
     for (int mt = 0; mt < kVEarly; ++mt)
       ldmatrix_x4_trans(vearly[mt], vt[mt & 3] + C::kBlkPitch * (mt >> 2));
-    if constexpr (QSPLIT) {
+    if constexpr (QSPLIT && DSPLIT == 2) {
       // each warp of the pair holds the scores over its half of D: exchange and add in
       // a fixed order (low half + high half) so both warps hold the same scores
 #pragma unroll
@@ -593,6 +595,24 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
           sc[nt][0] = t.x + sc[nt][0]; sc[nt][1] = t.y + sc[nt][1];
           sc[nt][2] = t.z + sc[nt][2]; sc[nt][3] = t.w + sc[nt][3];
         }
+      }
+    } else if constexpr (QSPLIT) {
+      // a quad: every warp holds the scores over its quarter of D; all four partial
+      // scores are summed in the order of the quarters, so every warp holds the same sums
+#pragma unroll
+      for (int nt = 0; nt < TPW; ++nt)
+        sXchg[((wslot * DSPLIT + wd) * TPW + nt) * 32 + lane] =
+            make_float4(sc[nt][0], sc[nt][1], sc[nt][2], sc[nt][3]);
+      named_barrier_sync(1 + wslot, 32 * DSPLIT);
+#pragma unroll
+      for (int nt = 0; nt < TPW; ++nt) {
+        float4 a = sXchg[((wslot * DSPLIT) * TPW + nt) * 32 + lane];
+#pragma unroll
+        for (int w = 1; w < DSPLIT; ++w) {
+          const float4 b = sXchg[((wslot * DSPLIT + w) * TPW + nt) * 32 + lane];
+          a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        sc[nt][0] = a.x; sc[nt][1] = a.y; sc[nt][2] = a.z; sc[nt][3] = a.w;
       }
     }
     float x[TPW][4];
@@ -1041,6 +1061,9 @@ constexpr int64_t kShape16MinWaves = 8;
 #ifndef QSA_SMALL16_CTAS
 #define QSA_SMALL16_CTAS 3
 #endif
+#ifndef QSA_SMALL16_DSPLIT
+#define QSA_SMALL16_DSPLIT 2  // warps of a slot lane splitting D: a pair (2) or a quad (4)
+#endif
 // E4M3 caches in such launches: one slot lane (a warp pair) of two stages, 25 KB, eight
 // CTAs per SM (long prefill 1.495 ms; two lanes of two stages at three or four CTAs 1.595,
 // of four stages 1.738; one lane of three stages at six CTAs 1.684, of four at five 1.749)
@@ -1056,7 +1079,7 @@ constexpr int64_t kShape16MinWaves = 8;
 #ifndef QSA_LARGE16_CTAS
 #define QSA_LARGE16_CTAS 3
 #endif
-using CfgSmall16 = Cfg<1, QSA_SMALL_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES, false, true>;
+using CfgSmall16 = Cfg<1, QSA_SMALL16_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES, false, true>;
 using CfgSmall8r16 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true, true>;
 using CfgSmall8s16 = Cfg<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES, true, true>;
 static_assert(CfgSmall16::kSmem <= CfgSmall16::kSmPerCta(QSA_SMALL16_CTAS), "16-bit shape: CTAs per SM");
@@ -1132,8 +1155,8 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
                      kLargeQsplit, true>(p, stream);
   } else {
     if (p.G <= 8)
-      e = shape16 ? launch_gather<1, 2, QSA_SMALL16_SL, QSA_SMALL16_STAGES, QSA_SMALL16_CTAS,
-                                  QSA_SMALL_QSPLIT, false, true>(p, stream, tma)
+      e = shape16 ? launch_gather<1, QSA_SMALL16_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES,
+                                  QSA_SMALL16_CTAS, QSA_SMALL_QSPLIT, false, true>(p, stream, tma)
                   : launch_gather<1, 2, QSA_SMALL_SL, QSA_SMALL_STAGES, QSA_SMALL_CTAS,
                                   QSA_SMALL_QSPLIT, false>(p, stream, tma);
     else if (shape16 && p.G <= QSA_LARGE16_QROWS)

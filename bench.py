@@ -45,6 +45,7 @@ WORKLOADS = {
     "tiny": lambda: wl.tiny(),
     "width_sweep": lambda: wl.width_sweep(),
     "causal_two_request": lambda: wl.causal_two_request(),
+    "causal_two_request_e4m3kv": lambda: wl.with_e4m3_cache(wl.causal_two_request()),
     "max_extent_g6_uniform": lambda: wl.max_extent(6, False),
     "max_extent_g6_clustered": lambda: wl.max_extent(6, True),
     "max_extent_g3_uniform": lambda: wl.max_extent(3, False),

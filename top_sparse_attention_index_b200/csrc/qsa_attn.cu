@@ -1079,6 +1079,23 @@ constexpr int64_t kShape16MinWaves = 8;
 #ifndef QSA_LARGE16_CTAS
 #define QSA_LARGE16_CTAS 3
 #endif
+// E4M3 caches, 8 < G <= 16, many-wave launches on caches of at most 65,536 rows: one slot
+// lane of three stages (the merge buffer of two head tiles needs the third), 37 KB, six
+// CTAs per SM (the causal batch with an E4M3 cache 4.005 vs 4.571 ms with the two-CTA
+// shape of three lanes of four stages; one lane of three stages at five CTAs 4.081, of
+// four stages at five 4.320, two lanes of four stages at two 4.961)
+#ifndef QSA_FP8_LARGE16
+#define QSA_FP8_LARGE16 1
+#endif
+#ifndef QSA_FP8_LARGE16_SL
+#define QSA_FP8_LARGE16_SL 1
+#endif
+#ifndef QSA_FP8_LARGE16_STAGES
+#define QSA_FP8_LARGE16_STAGES 3
+#endif
+#ifndef QSA_FP8_LARGE16_CTAS
+#define QSA_FP8_LARGE16_CTAS 6
+#endif
 using CfgSmall16 = Cfg<1, QSA_SMALL16_DSPLIT, QSA_SMALL16_SL, QSA_SMALL16_STAGES, false, true>;
 using CfgSmall8r16 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true, true>;
 using CfgSmall8s16 = Cfg<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES, true, true>;
@@ -1147,6 +1164,11 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
                                    true, true, true>(p, stream, tma)
                    : launch_gather<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS,
                                    true, true>(p, stream, tma);
+#if QSA_FP8_LARGE16
+    else if (shape16)
+      e = launch_gather<2, 2, QSA_FP8_LARGE16_SL, QSA_FP8_LARGE16_STAGES, QSA_FP8_LARGE16_CTAS,
+                        true, true, true>(p, stream, tma);
+#endif
     else if constexpr (QSA_LARGE_DSPLIT == 2)
       e = launch_gather<2, 2, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, QSA_LARGE_CTAS, true,
                         true>(p, stream, tma);

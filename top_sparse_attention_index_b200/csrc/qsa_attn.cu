@@ -998,6 +998,9 @@ cudaError_t launch_gather(const FwdParams& p, cudaStream_t stream, bool use_tma)
 #ifndef QSA_SMALL_CTAS
 #define QSA_SMALL_CTAS 2  // CTAs resident per SM
 #endif
+#ifndef QSA_FP8_SMALL_CTAS
+#define QSA_FP8_SMALL_CTAS 2
+#endif
 #ifndef QSA_LARGE_SL
 #define QSA_LARGE_SL 3
 #endif
@@ -1038,7 +1041,7 @@ using CfgSmall8 = Cfg<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, true>;
 using CfgLarge8 = Cfg<2, QSA_LARGE_DSPLIT, QSA_FP8_LARGE_SL, QSA_FP8_LARGE_STAGES, true>;
 static_assert(CfgSmall::kSmem <= CfgSmall::kSmPerCta(QSA_SMALL_CTAS), "small shape: CTAs per SM");
 static_assert(CfgLarge::kSmem <= CfgLarge::kSmPerCta(QSA_LARGE_CTAS), "large shape: CTAs per SM");
-static_assert(CfgSmall8::kSmem <= CfgSmall8::kSmPerCta(QSA_SMALL_CTAS), "E4M3 small shape: CTAs per SM");
+static_assert(CfgSmall8::kSmem <= CfgSmall8::kSmPerCta(QSA_FP8_SMALL_CTAS), "E4M3 small shape: CTAs per SM");
 static_assert(CfgLarge8::kSmem <= CfgLarge8::kSmPerCta(QSA_LARGE_CTAS), "E4M3 large shape: CTAs per SM");
 
 // Caches of at most 65,536 rows (the long prefill's among them): the compacted row list is
@@ -1051,7 +1054,10 @@ static_assert(CfgLarge8::kSmem <= CfgLarge8::kSmPerCta(QSA_LARGE_CTAS), "E4M3 la
 // caches take a shape of their own there (below; with fewer waves they keep four lanes of
 // three stages, with the 16-bit list).
 constexpr int64_t kRows16 = 65536;
-constexpr int64_t kShape16MinWaves = 8;
+#ifndef QSA_SHAPE16_MIN_WAVES
+#define QSA_SHAPE16_MIN_WAVES 8
+#endif
+constexpr int64_t kShape16MinWaves = QSA_SHAPE16_MIN_WAVES;
 #ifndef QSA_SMALL16_SL
 #define QSA_SMALL16_SL 2
 #endif
@@ -1117,7 +1123,7 @@ static_assert(CfgSmall8s16::kSmem <= CfgSmall8s16::kSmPerCta(QSA_FP8_SMALL16_CTA
 using CfgLarge16 = Cfg<2, 2, QSA_LARGE16_SL, QSA_LARGE16_STAGES, false, true, QSA_LARGE16_QROWS>;
 static_assert(CfgLarge16::kSmem <= CfgLarge16::kSmPerCta(QSA_LARGE16_CTAS),
               "12-row two-tile shape: CTAs per SM");
-static_assert(CfgSmall8r16::kSmem <= CfgSmall8r16::kSmPerCta(QSA_SMALL_CTAS),
+static_assert(CfgSmall8r16::kSmem <= CfgSmall8r16::kSmPerCta(QSA_FP8_SMALL_CTAS),
               "E4M3 16-bit shape: CTAs per SM");
 
 }  // namespace
@@ -1160,9 +1166,9 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
     if (p.G <= 8)
       e = shape16 ? launch_gather<1, 2, QSA_FP8_SMALL16_SL, QSA_FP8_SMALL16_STAGES,
                                   QSA_FP8_SMALL16_CTAS, true, true, true>(p, stream, tma)
-          : rows16 ? launch_gather<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS,
+          : rows16 ? launch_gather<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_FP8_SMALL_CTAS,
                                    true, true, true>(p, stream, tma)
-                   : launch_gather<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_SMALL_CTAS,
+                   : launch_gather<1, 2, QSA_FP8_SMALL_SL, QSA_FP8_SMALL_STAGES, QSA_FP8_SMALL_CTAS,
                                    true, true>(p, stream, tma);
 #if QSA_FP8_LARGE16
     else if (shape16)

@@ -512,9 +512,11 @@ __global__ void __launch_bounds__(32 * (DSPLIT > 1 ? DSPLIT : NTILE) * SL, MINB)
     if constexpr (TMA) {
       // the stage's K and V rows of both warps have landed (use s / STAGES of the buffer);
       // a bounded wait: on a time-out the error bit is set, later waits are skipped and
-      // the rows' outputs are not valid, but no warp leaves the pair's barriers
-      if (!tma_failed && !mbar_wait(full_bar(wslot, buf), (s / STAGES) & 1, kMaxPolls))
-        tma_failed = true;
+      // the rows' outputs are not valid, but no warp leaves the pair's barriers (the
+      // lanes agree on the outcome, so the warp stays converged)
+      const bool landed =
+          !tma_failed && mbar_wait(full_bar(wslot, buf), (s / STAGES) & 1, kMaxPolls);
+      if (!__all_sync(0xffffffffu, landed)) tma_failed = true;
     }
 
     // S^T (16 slots x 8 heads) = K (16 x 256) * Q^T (256 x 8) per head tile; each K

@@ -200,7 +200,8 @@ __global__ void __launch_bounds__(512, 1)
     int it = 0;
     for (; it < p.iters; ++it) {
       const int s = it % STAGES;
-      if (!mbar_wait(full(cw, s), (it / STAGES) & 1, kMaxPolls)) {
+      // every lane waits; the warp acts on the outcome as one (no lane leaves alone)
+      if (!__all_sync(0xffffffffu, mbar_wait(full(cw, s), (it / STAGES) & 1, kMaxPolls))) {
         failed = true;
         break;
       }
@@ -223,7 +224,8 @@ __global__ void __launch_bounds__(512, 1)
     int it = 0;
     for (; it < p.iters; ++it) {
       const int s = it % STAGES;
-      if (!mbar_wait(full(cw, s), (it / STAGES) & 1, kMaxPolls)) {
+      // every lane waits; the warp acts on the outcome as one (no lane leaves alone)
+      if (!__all_sync(0xffffffffu, mbar_wait(full(cw, s), (it / STAGES) & 1, kMaxPolls))) {
         failed = true;
         break;
       }
@@ -261,7 +263,7 @@ __global__ void __launch_bounds__(512, 1)
       uint32_t hv = p.seed ^ (0x9e3779b9u * (blockIdx.x * p.warps + cw + 1));
       for (int it = 0; it < p.iters; ++it) {
         const int s = it % STAGES;
-        if (!mbar_wait(full(cw, s), (it / STAGES) & 1, kMaxPolls)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(full(cw, s), (it / STAGES) & 1, kMaxPolls))) {
           failed = true;
           break;
         }

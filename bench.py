@@ -114,7 +114,11 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region.
+
+    A reader thread collects the samples; entering waits (up to 5 s) until the first
+    sample has arrived, so that even a timed region of a few tens of milliseconds falls
+    inside the sampled span."""
 
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -125,8 +129,16 @@ class ClockSampler:
         ids = [x.strip() for x in vis.split(",")] if vis else []
         self.gpu_index = ids[gpu_index] if gpu_index < len(ids) else str(gpu_index)
         self.proc = None
+        self.lines = []
+        self._thread = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.lines.append(line)
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
@@ -134,18 +146,26 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+        t_end = time.time() + 5.0
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
+            time.sleep(0.05)  # a sample after the end of the timed region
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                self.proc.wait()
+            if self._thread is not None:
+                self._thread.join(timeout=5)
 
     def summary(self, t0=None, t1=None):
         """Median SM clock and the throttle reasons seen between wall times t0 and t1."""
@@ -318,7 +338,6 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
-        time.sleep(0.3)  # let the sampler start
         t0_epoch = time.time()
         t_wall = time.perf_counter()
         for i in range(args.steps):

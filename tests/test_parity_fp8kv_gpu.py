@@ -340,3 +340,22 @@ def test_many_wave_launches_with_masks_and_splits(cuda_device, oracle_lib, Hq, H
     rows = sorted(set(range(0, Tq, 7)) | {1, 5, Tq - 1})
     compare(w, got, oracle_lib, 1.0 / 16.0, rows, f"E4M3 many waves Hq={Hq} S={S} nsplit={nsplit}")
     assert torch.all(got[5] == 0)
+
+
+def test_many_wave_two_tile_shape_block_and_shards(cuda_device, oracle_lib):
+    """The E4M3 shape for 8 < G <= 16 in many-wave launches (one slot lane, six CTAs per
+    SM) with block selection (block 4), and as context-parallel shards (R = 3, bf16
+    records) stacked and combined: every 9th row plus the first and last against the
+    oracle's fp8 path."""
+    from test_parity_gpu import _shards_combined
+    Tq, Hq, Hkv, S, W = 4000, 12, 1, 16384, 150
+    w = _random_case(2900, Tq, Hq, Hkv, S, W, minus1=0.1, widths=True)
+    w.slot_idx = wl.uniform_distinct(torch.Generator().manual_seed(2901), Tq, S // 4, W)
+    w.slot_idx[torch.rand(Tq, W, generator=torch.Generator().manual_seed(2902)) < 0.1] = -1
+    w.block = 4
+    rows = sorted(set(range(0, Tq, 9)) | {Tq - 1})
+    got = run(w, dev(w, cuda_device), 1.0 / 16.0)
+    compare(w, got, oracle_lib, 1.0 / 16.0, rows, "e4m3 two-tile many waves block4")
+    got, _ = _shards_combined(w, dev(w, cuda_device), 3, k_scale=w.k_scale, v_scale=w.v_scale,
+                              record_dtype=torch.bfloat16)
+    compare(w, got, oracle_lib, 1.0 / 16.0, rows, "e4m3 two-tile many waves block4, 3 shards")

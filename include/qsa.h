@@ -248,8 +248,21 @@ qsa_status_t qsa_sparse_prefill_fp8kv(const void* q, int64_t q_stride_t, int64_t
  *                      the base-2 log-sum-exp of the scaled scores; -inf where none.
  *                      Always fp32.
  *   record_bf16        0: part_o fp32; 1: part_o bf16.  Any other value: QSA_ERR_INVALID_ARG.
- * The split plan and workspace are those of qsa_sparse_prefill_block_plan; the device's
- * own splits are combined into the one record before the call's work ends.
+ * The split plan is that of qsa_sparse_prefill_block_plan, and so is the workspace the
+ * call requires; the device's own splits are combined into the one record before the
+ * call's work ends.  With an unsplit plan on a shard smaller than the whole cache
+ * (S < S_total), a workspace of the size qsa_sparse_prefill_partial_plan returns lets
+ * the call first copy every row's local entries (in order) to the workspace, so that the
+ * fused kernel reads only those instead of the whole global selection; with less (or
+ * none) the fused kernel scans the global selection itself.  Both give the same result,
+ * bit for bit.
+ *
+ * qsa_sparse_prefill_partial_plan: host only, like qsa_sparse_prefill_block_plan, whose
+ * split count it returns; *workspace_bytes (may be NULL) receives the workspace for the
+ * fastest form of the call: the split workspace when the plan splits W, else the
+ * compaction buffer ([Tq, W] and [Tq] int32, each 256-byte aligned) when the shard is
+ * smaller than the cache (S < S_total) and W >= 32, else 0.  Returns a negative
+ * qsa_status_t value for an invalid shape or 0 <= S <= S_total violated.
  *
  * qsa_combine_partials: out[t, h, :] = sum_r 2^(lse_r - m) O_r / sum_r 2^(lse_r - m),
  * m = max_r lse_r, over R records stacked as part_o [R, Tq, Hq, D] (fp32, or bf16 with
@@ -271,6 +284,11 @@ qsa_status_t qsa_sparse_prefill_partial(const void* q, int64_t q_stride_t, int64
                                         float* part_lse, int32_t record_bf16, int32_t nsplit,
                                         void* workspace, size_t workspace_bytes,
                                         uint32_t* err_word, void* stream);
+
+int32_t qsa_sparse_prefill_partial_plan(int32_t Tq, int32_t Hq, int32_t Hkv, int32_t D, int32_t W,
+                                        int32_t block, int64_t S, int64_t S_total,
+                                        int32_t num_sms, int32_t nsplit_request,
+                                        size_t* workspace_bytes);
 
 qsa_status_t qsa_combine_partials(const void* part_o, const float* part_lse, int32_t record_bf16,
                                   int32_t R, int32_t Tq, int32_t Hq, int32_t D, void* out,

@@ -349,3 +349,21 @@ def test_probe_valid_arguments_reach_the_device(lib):
     # without a GPU the first CUDA call fails: the arguments themselves were accepted
     st = qsa.qsa_probe_gather(1, 1, 0x1000, 1024, 512, 512, 4, 2, 8, 4, 1, 0x2000, None)
     assert st == qsa.QSA_ERR_CUDA
+
+
+def test_partial_plan_workspace(lib):
+    """A shard smaller than the cache with an unsplit plan asks for the compaction buffer
+    ([Tq, W] and [Tq] int32, each 256-byte aligned); the whole cache, a narrow selection
+    or a split plan ask for what qsa_sparse_prefill_block_plan asks for."""
+    def r256(x):
+        return (x + 255) // 256 * 256
+    n, ws = qsa.qsa_sparse_prefill_partial_plan(7810, 16, 2, 256, 2051, 1, 8192, 65536, 148)
+    assert n == 1 and ws == r256(7810 * 2051 * 4) + r256(7810 * 4)
+    assert qsa.qsa_sparse_prefill_partial_plan(7810, 16, 2, 256, 2051, 1, 65536, 65536, 148) == (1, 0)
+    assert qsa.qsa_sparse_prefill_partial_plan(100, 16, 2, 256, 31, 1, 10, 100, 148) == (1, 0)
+    split = qsa.qsa_sparse_prefill_partial_plan(4, 16, 2, 256, 2051, 1, 8192, 65536, 148)
+    assert split == qsa.qsa_sparse_prefill_block_plan(4, 16, 2, 256, 2051, 1, 148) and split[0] > 1
+    for S, S_total in ((10, 5), (-1, 5)):
+        with pytest.raises(qsa.QSAError) as ei:
+            qsa.qsa_sparse_prefill_partial_plan(4, 16, 2, 256, 64, 1, S, S_total, 148)
+        assert ei.value.status == qsa.QSA_ERR_INVALID_ARG

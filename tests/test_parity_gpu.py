@@ -668,6 +668,40 @@ def test_context_parallel_shards(cuda_device, oracle_lib, R, rec):
         assert all((o[t] == 0).all() for o in _shards_combined.last_records)
 
 
+def test_context_parallel_compaction_is_bitwise_the_full_scan(cuda_device):
+    """A shard given the workspace for the compaction pass (every row's local entries
+    copied first) returns bitwise the record of the same shard scanning the global
+    selection itself, and flags the same invalid values: ragged widths (some outside
+    [0, W]), interior -1, out-of-range slots, rows with no local entry; block selection
+    too."""
+    for block, R in ((1, 3), (4, 5)):
+        w = _random_case(480 + block, 700, 16, 2, 16384, 2051 // block, minus1=0.1, widths=True)
+        w.block = block
+        w.slot_idx = wl.uniform_distinct(torch.Generator().manual_seed(481), 700, 16384 // block,
+                                         2051 // block)
+        w.slot_idx[torch.rand(700, 2051 // block, generator=torch.Generator().manual_seed(482)) < 0.1] = -1
+        w.slot_idx[7, 3] = 16384 // block + 5          # invalid: past the cache
+        w.slot_idx[8, 0] = -7                          # invalid: negative
+        w.width[7] = w.width[8] = 2051 // block        # (both read)
+        w.width[9] = 2051 // block + 3                 # invalid: width past W
+        w.width[10] = -2                               # invalid: negative width
+        d = dev(w, cuda_device)
+        for lo, hi in qsa.shard_ranges(w.S, R, block):
+            recs, errs = [], []
+            for compact in (True, False):
+                err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+                po, pl = qsa.sparse_prefill_partial(d["q"], d["k_cache"][lo:hi], d["v_cache"][lo:hi],
+                                                    d["slot_idx"], lo, w.S, width=d["width"],
+                                                    block=block, err_word=err, compact=compact,
+                                                    record_dtype=torch.bfloat16)
+                torch.cuda.synchronize()
+                recs.append((po.cpu(), pl.cpu()))
+                errs.append(int(err.item()))
+            assert torch.equal(recs[0][0].view(torch.int16), recs[1][0].view(torch.int16))
+            assert torch.equal(recs[0][1], recs[1][1])
+            assert errs[0] == errs[1] == 3, errs
+
+
 def test_context_parallel_wide_rows_and_decode(cuda_device, oracle_lib):
     """W = 6,000 (each shard combines its own splits into one record) and a decode-shape
     batch with forced split counts."""

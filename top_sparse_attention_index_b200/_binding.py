@@ -47,6 +47,8 @@ SIGNATURES = {
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _i32,
                                           _i64, _i64, _i32, _f, _f, _f, _p, _p, _i32, _i32, _p,
                                           _sz, _p, _p]),
+    "qsa_sparse_prefill_partial_plan": (_i32, [_i32, _i32, _i32, _i32, _i32, _i32, _i64, _i64,
+                                               _i32, _i32, ctypes.POINTER(_sz)]),
     "qsa_combine_partials": (_i32, [_p, _p, _i32, _i32, _i32, _i32, _i32, _p, _i64, _i64, _p]),
     "qsa_sparse_prefill_noalloc": (_i32, [_p, _i64, _i64, _p, _i64, _i64, _p, _i64, _i64, _p,
                                           _i64, _p, _i32, _i32, _i32, _i32, _i64, _i32, _f, _p,
@@ -186,6 +188,19 @@ def qsa_sparse_prefill_partial(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k
         part_lse, record_bf16, nsplit, workspace, workspace_bytes, err_word, stream))
 
 
+def qsa_sparse_prefill_partial_plan(Tq, Hq, Hkv, D, W, block, S, S_total, num_sms,
+                                    nsplit_request=0):
+    """(nsplit, workspace_bytes) of a slot-range shard's call; raises QSAError for invalid
+    shapes."""
+    ws = ctypes.c_size_t(0)
+    n = int(load_library().qsa_sparse_prefill_partial_plan(Tq, Hq, Hkv, D, W, block, S, S_total,
+                                                           num_sms, nsplit_request,
+                                                           ctypes.byref(ws)))
+    if n < 0:
+        raise QSAError(-n, qsa_last_error_detail())
+    return n, int(ws.value)
+
+
 def qsa_combine_partials(part_o, part_lse, record_bf16, R, Tq, Hq, D, out, out_stride_t,
                          out_stride_h, stream) -> int:
     """Raw call of the log-sum-exp combine of R stacked partial records."""
@@ -282,7 +297,7 @@ def sparse_prefill(q, k_cache, v_cache, slot_idx, width=None, scale=None, out=No
 def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, width=None,
                            scale=None, part_o=None, part_lse=None, nsplit=0, err_word=None,
                            stream=None, block=1, k_scale=1.0, v_scale=1.0,
-                           record_dtype=torch.float32):
+                           record_dtype=torch.float32, compact=True):
     """One device's partial record for a cache split by slot range (context parallel).
 
     k_cache / v_cache hold the global slots [slot_lo, slot_lo + S) of a cache of S_total
@@ -290,7 +305,9 @@ def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, widt
     slot numbers.  Returns (part_o [Tq, Hq, 256] of record_dtype (float32 or bfloat16),
     part_lse fp32 [Tq, Hq]): the output normalised over this device's valid slots and the
     base-2 log-sum-exp of their scaled scores (-inf where there are none).  Combine the
-    records of all devices with combine_partials.
+    records of all devices with combine_partials.  compact=True gives the call the
+    workspace in which it first gathers each row's local entries (same result, fewer
+    entries for the fused kernel to scan); False gives it only the split workspace.
     """
     device = q.device
     if device.type != "cuda":
@@ -324,7 +341,11 @@ def sparse_prefill_partial(q, k_cache, v_cache, slot_idx, slot_lo, S_total, widt
     if stream is None:
         stream = torch.cuda.current_stream(device)
     num_sms = torch.cuda.get_device_properties(device).multi_processor_count
-    ns, ws_bytes = qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, block, num_sms, nsplit)
+    if compact:
+        ns, ws_bytes = qsa_sparse_prefill_partial_plan(Tq, Hq, Hkv, D, W, block, S,
+                                                       int(S_total), num_sms, nsplit)
+    else:
+        ns, ws_bytes = qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, D, W, block, num_sms, nsplit)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device) if ws_bytes else None
     with torch.cuda.device(device):
         st = qsa_sparse_prefill_partial(

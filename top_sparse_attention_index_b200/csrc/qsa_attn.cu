@@ -918,6 +918,53 @@ __global__ void __launch_bounds__(128) qsa_lse_combine_kernel(const FwdParams p)
   if (p.partial_out && lane == 0) p.part_lse[row] = mstar + fast_log2(wsum);
 }
 
+// Shard compaction (context parallelism): one warp per query row reads the row's selected
+// entries (up to its width, clamped as K1 does) 32 at a time, flags invalid values, and
+// appends the entries held by this shard in their original order (a ballot and a prefix
+// count per 32 entries).  K1 then runs on the compacted rows with the counts as widths and
+// sees exactly the local entries it would have kept itself, in the same order.
+__global__ void __launch_bounds__(128) qsa_shard_compact_kernel(const FwdParams p, int32_t* idx,
+                                                                int32_t* count) {
+  const int64_t t = int64_t(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  if (t >= p.Tq) return;
+  const int lane = threadIdx.x & 31;
+  int wv = p.W;
+  if (p.width != nullptr) {
+    wv = p.width[t];
+    if (wv < 0 || wv > p.W) {
+      if (lane == 0 && p.err_word != nullptr) atomicOr(p.err_word, 2u);
+      wv = wv < 0 ? 0 : p.W;
+    }
+  }
+  const int32_t* src = p.slot_idx + t * p.idx_stride_t;
+  int32_t* dst = idx + t * int64_t(p.W);
+  const uint32_t ent_lo = uint32_t(p.ent_lo), ent_n = uint32_t(p.ent_hi - p.ent_lo);
+  const uint32_t below = (1u << lane) - 1u;
+  // 256 entries per step: each lane's eight loads are in flight together, then the eight
+  // 32-entry groups are appended in order
+  constexpr int kUnroll = 8;
+  int n = 0;
+  bool bad = false;
+  for (int base = 0; base < wv; base += 32 * kUnroll) {
+    int v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i = base + 32 * u + lane;
+      v[u] = i < wv ? __ldg(src + i) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      bad |= v[u] != -1 && uint32_t(v[u]) >= uint32_t(p.ent_total);
+      const bool loc = uint32_t(v[u]) - ent_lo < ent_n;
+      const uint32_t m = __ballot_sync(0xffffffffu, loc);
+      if (loc) dst[n + __popc(m & below)] = v[u];
+      n += __popc(m);
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && p.err_word != nullptr) atomicOr(p.err_word, 1u);
+  if (lane == 0) count[t] = n;
+}
+
 template <int NTILE, int DSPLIT, int SL, int STAGES, int MINB, bool QSPLIT, bool KV8,
           bool SLOT16 = false, int QROWS = NTILE * 8, bool TMA = false>
 cudaError_t launch_fwd(const FwdParams& p, cudaStream_t stream) {
@@ -1201,6 +1248,19 @@ cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   }
   if (e != cudaSuccess || p.nsplit == 1) return e;
   return launch_combine(p, stream);
+}
+
+size_t shard_compact_bytes(int32_t Tq, int32_t W) {
+  const size_t idx_bytes = (size_t(Tq) * size_t(W) * 4 + 255) / 256 * 256;
+  return idx_bytes + (size_t(Tq) * 4 + 255) / 256 * 256;
+}
+
+cudaError_t launch_shard_compact(const FwdParams& p, int32_t* idx, int32_t* count,
+                                 cudaStream_t stream) {
+  if (p.Tq == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((int64_t(p.Tq) + 3) / 4);
+  qsa_shard_compact_kernel<<<grid, 128, 0, stream>>>(p, idx, count);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream) {

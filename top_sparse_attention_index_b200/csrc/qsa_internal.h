@@ -96,6 +96,13 @@ cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream);
 
 size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit);
 
+// Context-parallel shards: a pass that copies every row's local entries (in order, after
+// the width and validity checks) to idx [Tq, W] (row stride W) and their number to
+// count [Tq], so that K1 then reads only those.  Scratch: the two arrays, 256-aligned.
+size_t shard_compact_bytes(int32_t Tq, int32_t W);
+cudaError_t launch_shard_compact(const FwdParams& p, int32_t* idx, int32_t* count,
+                                 cudaStream_t stream);
+
 // printf-style detail for qsa_last_error_detail() on the calling host thread.
 void set_error_detail(const char* fmt, ...);
 

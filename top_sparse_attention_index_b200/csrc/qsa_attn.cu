@@ -6,14 +6,16 @@
 // scale * Q K^T for the whole GQA group of G = Hq / Hkv query heads, take the softmax
 // over the selected slots only and return P V; a row without a valid slot returns 0.
 //
-// K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit, two or three CTAs
+// K1 qsa_sparse_attn_fwd_kernel -- one CTA per (t, j, split) work unit, several CTAs
 // resident per SM so that one CTA's prologue and epilogue overlap the others' gathers
-// (three, of two slot lanes each, when the cache has at most 65,536 rows so the compacted
-// row list is 16-bit, and the launch has many waves; units ordered KV head slowest when
-// one head's slice of the cache fits L2 and the whole cache does not):
+// (bf16: two, or three of two slot lanes each when the cache has at most 65,536 rows so
+// the compacted row list is 16-bit and the launch has many waves; E4M3 caches in such
+// launches: eight of one slot lane for G <= 8, six for G > 8; units ordered KV head
+// slowest when one head's slice of the cache fits L2 and the whole cache does not):
 //   1. stage the split's slot indices in shared memory and compact away -1 (and
 //      out-of-range) entries with a block scan, so masked slots cost no bandwidth;
-//   2. gather K and V rows of the compacted slots with 16-byte cp.async into shared
+//   2. gather K and V rows of the compacted slots with 16-byte cp.async (or, in builds
+//      that ask for it, TMA tile::gather4, measured slower) into shared
 //      memory: each 16-slot sub-tile of a stage belongs to one slot lane (a warp pair)
 //      that loads it, waits for it and consumes it, so the lanes run STAGES-deep
 //      pipelines of their own with no block-wide barrier in the loop (row = 512
@@ -29,7 +31,10 @@
 //   4. merge the per-warp (m, l, O) states through shared memory and write bf16 out
 //      (exact zeros for empty rows), or fp32 partials + base-2 LSE when split.
 // K2 qsa_lse_combine_kernel -- one warp per (t, h): log-sum-exp weighted sum of the
-//   split partials; empty splits carry LSE = -inf and weight 0; all empty -> exact 0.
+//   split partials (or of context-parallel records, fp32 or bf16); empty splits carry
+//   LSE = -inf and weight 0; all empty -> exact 0.
+// qsa_shard_compact_kernel -- context-parallel shards: each row's local entries copied in
+//   order before K1, which then scans only those.
 //
 // fp8_e4m3 KV cache (the format named in section "Where this sits in the Qwen4Exp serving
 // build-out" of the same article): K1 with KV8 gathers 256-byte rows of E4M3 codes (half

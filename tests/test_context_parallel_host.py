@@ -144,3 +144,112 @@ def test_shard_ranges_cover_the_cache_once():
         assert len(r) == world and r[0][0] == 0 and r[-1][1] == S
         assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
         assert all(hi >= lo and (lo % block == 0 or hi == lo) for lo, hi in r)
+
+
+# ---- the peer exchange (records read in place, outputs stored to every rank) -------------
+
+class _FakeIPC:
+    """Stands in for the CUDA IPC helpers on the CPU: a handle names (rank, buffer number)
+    and an import returns a synthetic base address for it (never dereferenced)."""
+
+    def __init__(self, rank):
+        self.rank, self.n, self.opened, self.closed = rank, 0, [], []
+
+    def ipc_export(self, t):
+        self.n += 1
+        return bytes([self.rank, self.n]) + bytes(62), 16 * self.n
+
+    def ipc_import(self, handle, device):
+        base = ((1 + handle[0]) << 40) | (handle[1] << 32)
+        self.opened.append(base)
+        return base
+
+    def ipc_close(self, base, device):
+        self.closed.append(base)
+
+
+def _peer_combine_emulated(o_ptrs, lse_ptrs, record_dtype, Tq, Hq, outs, t0, t1, device=None):
+    """The peer combine restated on the CPU: the pointer table is checked against the
+    exchange's buffers; reading the other ranks' records in place is emulated by a gather,
+    and storing the rows [t0, t1) to every rank's output by a gather of the row blocks."""
+    import torch.distributed as dist
+    ex = next(iter(cp._EXCHANGES.values()))
+    for r in range(ex.world):
+        own = r == ex.rank
+        base = ((1 + r) << 40)
+        assert o_ptrs[r] == (ex.part_o.data_ptr() if own else (base | 1 << 32) + 16)
+        assert lse_ptrs[r] == (ex.part_lse.data_ptr() if own else (base | 2 << 32) + 32)
+        assert outs[r][0] == (ex.out.data_ptr() if own else (base | 3 << 32) + 48)
+    assert (t0, t1) == tuple(cp.shard_ranges(Tq, ex.world)[ex.rank])
+    g_o = [torch.empty_like(ex.part_o) for _ in range(ex.world)]
+    g_l = [torch.empty_like(ex.part_lse) for _ in range(ex.world)]
+    dist.all_gather(g_o, ex.part_o)
+    dist.all_gather(g_l, ex.part_lse)
+    rows = _combine_double(torch.stack(g_o)[:, t0:t1], torch.stack(g_l)[:, t0:t1])
+    blocks = [None] * ex.world
+    dist.all_gather_object(blocks, (t0, t1, rows.to(torch.bfloat16)))
+    for a, b, blk in blocks:
+        ex.out[a:b] = blk
+
+
+def _partial_into(q, k_local, v_local, slot_idx, slot_lo, S_total, part_o=None, part_lse=None,
+                  **kw):
+    o, lse = _partial_double(q, k_local, v_local, slot_idx, slot_lo, S_total, **kw)
+    part_o.copy_(o)
+    part_lse.copy_(lse)
+    return part_o, part_lse
+
+
+def _peer_rank_main(rank, world, port, queue):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    q, k, v, idx = _case()
+    S = k.shape[0]
+    lo, hi = cp.shard_ranges(S, world)[rank]
+    ipc = _FakeIPC(rank)
+    outs = []
+    for _ in range(2):  # the second call reuses the exchange (no new export or import)
+        outs.append(cp.sparse_prefill_context_parallel(
+            q, k[lo:hi], v[lo:hi], idx, lo, S, exchange="peer", partial_fn=_partial_into,
+            peer_combine_fn=_peer_combine_emulated, ipc=ipc, record_dtype=torch.bfloat16))
+    opened = list(ipc.opened)
+    cp.release_peer_exchanges()
+    queue.put((rank, [o.float().numpy() for o in outs], opened, list(ipc.closed), ipc.n))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_peer_exchange_protocol(oracle_lib):
+    """World sizes 2 and 3: every rank exports its three buffers once, maps the other ranks'
+    (one mapping per exported allocation), combines its own share of the rows, and ends
+    with the whole output; both calls give the whole-cache result (bf16 records and bf16
+    output: within 2^-8 of the largest |V|), the same on every rank; release unmaps exactly
+    what was mapped."""
+    q, k, v, idx = _case()
+    ref = oracle_lib.forward(q, k, v, idx, None, 1.0 / 16.0)
+    bound = 2.0 ** -8 * float(v.float().abs().max()) + 1e-6
+    for world in (2, 3):
+        ctx = mp.get_context("spawn")
+        queue = ctx.Queue()
+        port = _free_port()
+        procs = [ctx.Process(target=_peer_rank_main, args=(r, world, port, queue))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        results = {}
+        for _ in procs:
+            rank, outs, opened, closed, exported = queue.get(timeout=180)
+            results[rank] = outs
+            assert exported == 3
+            assert len(opened) == 3 * (world - 1) and sorted(closed) == sorted(opened)
+        for p in procs:
+            p.join(timeout=60)
+            assert p.exitcode == 0
+        for r in range(world):
+            for out in results[r]:
+                assert np.abs(out - ref).max() <= bound
+                np.testing.assert_array_equal(out, results[0][0])
+            assert np.all(results[r][0][1] == 0)   # the fully masked row

@@ -34,17 +34,25 @@ from ._binding import (  # noqa: F401
     qsa_sparse_prefill_workspace_bytes,
     qsa_status_string,
     combine_partials,
+    combine_peer_records,
+    qsa_combine_peer_records,
     sparse_prefill,
     sparse_prefill_from_host,
     sparse_prefill_partial,
 )
-from .context_parallel import shard_ranges, sparse_prefill_context_parallel  # noqa: F401
+from .context_parallel import (  # noqa: F401
+    PeerExchange,
+    release_peer_exchanges,
+    shard_ranges,
+    sparse_prefill_context_parallel,
+)
 
 __all__ = [
     "sparse_prefill", "sparse_prefill_from_host", "qsa_sparse_prefill", "qsa_sparse_prefill_noalloc",
     "qsa_sparse_prefill_block", "qsa_sparse_prefill_block_plan", "qsa_sparse_prefill_fp8kv",
     "qsa_sparse_prefill_partial", "qsa_sparse_prefill_partial_plan", "qsa_combine_partials", "sparse_prefill_partial",
     "combine_partials", "sparse_prefill_context_parallel", "shard_ranges",
+    "qsa_combine_peer_records", "combine_peer_records", "PeerExchange", "release_peer_exchanges",
     "qsa_sparse_prefill_plan", "qsa_sparse_prefill_workspace_bytes", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
     "load_library", "QSAError", "qsa_probe_gather",
 ]

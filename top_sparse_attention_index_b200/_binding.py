@@ -25,6 +25,8 @@ QSA_ERRBIT_Q_RANGE = 0x4
 QSA_MAX_SLOTS_PER_SPLIT = 2240
 QSA_MAX_BLOCK = 16
 QSA_STATIC_SCRATCH_BYTES = 16 << 20
+QSA_MAX_PEERS = 16
+QSA_IPC_HANDLE_BYTES = 64
 
 # Every symbol include/qsa.h declares, with its ctypes signature (restype, argtypes).
 _p, _i32, _i64, _sz, _f = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -55,6 +57,12 @@ SIGNATURES = {
                                           _i64, _i64, _i32, _p, _p]),
     "qsa_probe_gather": (_i32, [_i32, _i32, _p, _i64, _i64, _i32, _i32, _i32, _i32, _i32,
                                 ctypes.c_uint32, _p, _p]),
+    "qsa_combine_peer_records": (_i32, [ctypes.POINTER(_p), ctypes.POINTER(_p), _i32, _i32, _i32,
+                                        _i32, _i32, _i32, _i32, ctypes.POINTER(_p), _i32, _i64,
+                                        _i64, _p]),
+    "qsa_ipc_export": (_i32, [_p, _p, ctypes.POINTER(ctypes.c_uint64)]),
+    "qsa_ipc_import": (_i32, [_p, ctypes.POINTER(_p)]),
+    "qsa_ipc_close": (_i32, [_p]),
     "qsa_status_string": (ctypes.c_char_p, [_i32]),
     "qsa_last_error_detail": (ctypes.c_char_p, []),
 }
@@ -389,6 +397,98 @@ def combine_partials(part_o, part_lse, out=None, stream=None):
     if st != QSA_OK:
         raise QSAError(st, qsa_last_error_detail())
     return out
+
+
+# ---- records addressed one pointer each (include/qsa_peer.h) --------------------------
+
+def _ptr_array(ptrs):
+    arr = (ctypes.c_void_p * len(ptrs))()
+    for i, v in enumerate(ptrs):
+        arr[i] = int(v)
+    return arr
+
+
+def qsa_combine_peer_records(rec_o, rec_lse, R, record_bf16, Tq, Hq, D, t0, t1, out, n_out,
+                             out_stride_t, out_stride_h, stream) -> int:
+    """Raw call: rec_o, rec_lse and out are sequences of integer device pointers (the
+    host arrays of the C call); returns the status code."""
+    return int(load_library().qsa_combine_peer_records(
+        _ptr_array(rec_o), _ptr_array(rec_lse), R, record_bf16, Tq, Hq, D, t0, t1,
+        _ptr_array(out), n_out, out_stride_t, out_stride_h, stream))
+
+
+def combine_peer_records(rec_o_ptrs, rec_lse_ptrs, record_dtype, Tq, Hq, outs, t0=0, t1=None,
+                         stream=None, device=None):
+    """The log-sum-exp combine of R records given as device pointers (this device's memory
+    or peer memory mapped into this process), rows [t0, t1) stored as bf16 to every tensor
+    in `outs` (bf16 [Tq, Hq, 256] tensors, or (pointer, stride_t, stride_h) triples that
+    share the strides of the first).  Returns nothing; the work is enqueued on `stream`."""
+    device = torch.device(device) if device is not None else None
+    t1 = Tq if t1 is None else t1
+    if record_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("record_dtype must be torch.float32 or torch.bfloat16")
+    if len(rec_o_ptrs) != len(rec_lse_ptrs):
+        raise ValueError("one O pointer and one lse pointer per record")
+    out_ptrs, strides = [], None
+    for o in outs:
+        if isinstance(o, torch.Tensor):
+            _check_dev("out", o, torch.bfloat16, o.device)
+            if tuple(o.shape) != (Tq, Hq, 256):
+                raise ValueError("every out must be [Tq, Hq, 256]")
+            device = device or o.device
+            st = (o.stride(0), o.stride(1))
+            out_ptrs.append(_ptr(o))
+        else:
+            ptr, st_t, st_h = o
+            st = (st_t, st_h)
+            out_ptrs.append(int(ptr))
+        if strides is not None and st != strides:
+            raise ValueError("every out must have the same strides")
+        strides = st
+    if strides is None:
+        raise ValueError("at least one out")
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    with torch.cuda.device(device):
+        st = qsa_combine_peer_records(rec_o_ptrs, rec_lse_ptrs, len(rec_o_ptrs),
+                                      1 if record_dtype == torch.bfloat16 else 0, Tq, Hq, 256,
+                                      t0, t1, out_ptrs, len(out_ptrs), strides[0], strides[1],
+                                      stream.cuda_stream)
+    if st != QSA_OK:
+        raise QSAError(st, qsa_last_error_detail())
+
+
+def ipc_export(t: torch.Tensor):
+    """(handle bytes, byte offset) that let another process map the memory of `t`."""
+    h = ctypes.create_string_buffer(QSA_IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64(0)
+    with torch.cuda.device(t.device):
+        st = int(load_library().qsa_ipc_export(_ptr(t), h, ctypes.byref(off)))
+    if st != QSA_OK:
+        raise QSAError(st, qsa_last_error_detail())
+    return h.raw, int(off.value)
+
+
+def ipc_import(handle: bytes, device) -> int:
+    """Maps another process's exported allocation on `device`; returns its base pointer."""
+    if len(handle) != QSA_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is %d bytes" % QSA_IPC_HANDLE_BYTES)
+    base = ctypes.c_void_p(0)
+    with torch.cuda.device(device):
+        st = int(load_library().qsa_ipc_import(ctypes.create_string_buffer(handle, len(handle)),
+                                               ctypes.byref(base)))
+    if st != QSA_OK:
+        raise QSAError(st, qsa_last_error_detail())
+    return int(base.value)
+
+
+def ipc_close(base: int, device) -> None:
+    with torch.cuda.device(device):
+        st = int(load_library().qsa_ipc_close(ctypes.c_void_p(base)))
+    if st != QSA_OK:
+        raise QSAError(st, qsa_last_error_detail())
 
 
 _COPY_STREAMS = {}

@@ -73,6 +73,9 @@ class PeerExchange:
         import torch.distributed as dist
         self.group, self.device = group, torch.device(device)
         self.rank, self.world = dist.get_rank(group), dist.get_world_size(group)
+        if self.world > _binding.QSA_MAX_PEERS:
+            raise ValueError("the peer exchange serves at most %d ranks (got %d): use "
+                             'exchange="all_gather"' % (_binding.QSA_MAX_PEERS, self.world))
         self.Tq, self.Hq, self.record_dtype = Tq, Hq, record_dtype
         self._ipc = ipc or _binding
         dev = self.device
@@ -131,7 +134,8 @@ _EXCHANGES = {}
 
 
 def peer_exchange(group, device, Tq, Hq, record_dtype, ipc=None):
-    """The PeerExchange of this shape, created on first use (collectively) and kept."""
+    """The PeerExchange of this shape, created on first use (collectively) and kept until
+    release_peer_exchanges(), which every rank must call before the group is destroyed."""
     import torch.distributed as dist
     key = (id(group) if group is not None else None, dist.get_rank(group),
            torch.device(device), Tq, Hq, record_dtype)

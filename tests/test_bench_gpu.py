@@ -52,3 +52,20 @@ def test_reference_arm_line(cuda_device):
     d = _bench("--impl", "reference", "--steps", "1", "--warmup", "1")
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s"
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_context_parallel_bench_line(cuda_device):
+    """The context-parallel measurement (ranks emulated on one GPU) at a decode shape:
+    one JSON line whose per-R entries carry the shard, combine and link-byte figures."""
+    out = subprocess.run([sys.executable, "-m", "top_sparse_attention_index_b200.context_parallel_bench",
+                          "--rows", "64", "--ranks", "2,3", "--reps", "3"], cwd=ROOT,
+                         capture_output=True, text=True, timeout=900)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = json.loads([l for l in out.stdout.splitlines() if l.startswith("{")][-1])
+    assert d["unit"] == "us" and d["unsharded_us"] > 0
+    assert [(e["R"], e["record"]) for e in d["ranks"]] == [(2, "bfloat16"), (3, "bfloat16"),
+                                                           (2, "float32"), (3, "float32")]
+    for e in d["ranks"]:
+        assert len(e["shard_us"]) == e["R"] and e["shard_max_us"] == max(e["shard_us"])
+        assert e["all_gather_bytes_in_per_rank"] == (e["R"] - 1) * e["record_bytes_per_rank"]
+        assert e["peer_bytes_in_per_rank"] < e["all_gather_bytes_in_per_rank"]

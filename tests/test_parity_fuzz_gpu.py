@@ -97,3 +97,41 @@ def test_random_shapes_match_oracle(cuda_device, oracle_lib, seed):
     torch.cuda.synchronize()
     assert int(err.item()) == 0, label
     check_gates(out.cpu().float(), torch.from_numpy(ref), _empty_rows(c), label)
+
+
+@pytest.mark.parametrize("seed", range(7100, 7108))
+def test_random_context_parallel_shards_match_oracle(cuda_device, oracle_lib, seed):
+    """The same random draws split by slot range over 2-6 emulated ranks (shard boundaries
+    on block multiples), bf16 or fp32 records, combined both ways: stacked (as after an
+    all-gather) and through one pointer per record (as the peer exchange reads them).  The
+    two combines agree bitwise; the result meets the gates against the whole-cache oracle."""
+    c = _draw(seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    R = int(torch.randint(2, 7, (1,), generator=g))
+    rec = torch.bfloat16 if int(torch.randint(0, 2, (1,), generator=g)) else torch.float32
+    label = (f"seed {seed}: R={R} {rec} Tq={c['Tq']} Hq={c['Hq']} Hkv={c['Hkv']} S={c['S']} "
+             f"W={c['W']} block={c['block']} fp8={c['fp8']}")
+    if c["fp8"]:
+        ks, vs = wl.E4M3_K_SCALE, wl.E4M3_V_SCALE
+        k, v = wl.to_e4m3_cache(c["k"], ks), wl.to_e4m3_cache(c["v"], vs)
+        ref = oracle_lib.forward_fp8kv(c["q"], k, v, c["idx"], c["width"], c["scale"], ks, vs,
+                                       block=c["block"])
+    else:
+        ks = vs = 1.0
+        k, v = c["k"].to(torch.bfloat16), c["v"].to(torch.bfloat16)
+        ref = oracle_lib.forward(c["q"], k, v, c["idx"], c["width"], c["scale"], block=c["block"])
+    q = c["q"].contiguous().to(cuda_device)
+    kd, vd, idx = k.to(cuda_device), v.to(cuda_device), c["idx"].to(cuda_device)
+    width = None if c["width"] is None else c["width"].to(cuda_device)
+    recs = [qsa.sparse_prefill_partial(q, kd[lo:hi], vd[lo:hi], idx, lo, c["S"], width=width,
+                                       scale=c["scale"], block=c["block"], k_scale=ks,
+                                       v_scale=vs, record_dtype=rec)
+            for lo, hi in qsa.shard_ranges(c["S"], R, c["block"])]
+    stacked = qsa.combine_partials(torch.stack([r[0] for r in recs]),
+                                   torch.stack([r[1] for r in recs]))
+    peer = torch.empty_like(stacked)
+    qsa.combine_peer_records([r[0].data_ptr() for r in recs], [r[1].data_ptr() for r in recs],
+                             rec, c["Tq"], c["Hq"], [peer])
+    torch.cuda.synchronize()
+    assert torch.equal(peer.view(torch.int16), stacked.view(torch.int16)), label
+    check_gates(stacked.cpu().float(), torch.from_numpy(ref), _empty_rows(c), label)

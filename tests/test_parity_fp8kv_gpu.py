@@ -328,7 +328,7 @@ def test_cache_offsets_beyond_4gib(cuda_device, oracle_lib):
 @pytest.mark.parametrize("Hq,Hkv,S,nsplit", [(8, 2, 8192, 1), (6, 1, 30000, 3), (12, 1, 12000, 1),
                                               (24, 2, 12288, 2), (16, 1, 65536, 1)])
 def test_many_wave_launches_with_masks_and_splits(cuda_device, oracle_lib, Hq, Hkv, S, nsplit):
-    """E4M3 launches of many waves (at least eight waves of three CTAs per SM) on caches of
+    """E4M3 launches of many waves (at least four waves of three CTAs per SM) on caches of
     at most 65,536 rows, for G <= 8 and for 8 < G <= 16 (each has its own shape there):
     ragged widths, interior -1 entries, an empty row, one split and forced splits; the
     oracle's fp8 path checks every 7th row plus the first and last."""

@@ -178,7 +178,7 @@ def test_forced_splits_decode_shape(cuda_device, oracle_lib, nsplit):
                                              (6, 1, 20000, 3), (24, 2, 12288, 2), (20, 2, 4096, 1),
                                              (12, 1, 30000, 0), (32, 2, 8192, 1)])
 def test_many_wave_launches_with_masks_and_splits(cuda_device, oracle_lib, Hq, Hkv, S, nsplit):
-    """Launches of many waves (at least eight waves of three CTAs per SM) on caches of at
+    """Launches of many waves (at least five waves of three CTAs per SM) on caches of at
     most 65,536 rows, for one head tile (G <= 8), two tiles with the 12-row Q tile
     (G = 10, 12) and two tiles with the full one (G = 16): ragged widths, interior -1
     entries and empty rows, with one split, forced splits (partials and the combine) and

@@ -1109,15 +1109,20 @@ static_assert(CfgLarge8::kSmem <= CfgLarge8::kSmPerCta(QSA_LARGE_CTAS), "E4M3 la
 // (12 warps, as before) fit on an SM and hide one another's per-unit prologue and epilogue
 // better than two CTAs of three lanes (measured: long prefill 2.016 vs 2.096 ms, 512-slot
 // rows 0.317 vs 0.356 ms).  A CTA of two lanes takes ~1.4x as long per unit, so with few
-// units the coarser waves lose (4,000 units: 0.557 vs 0.564 ms; 2,048: 0.303 vs 0.297;
-// 512: 140 vs 102 us): the shape is used from eight waves of three CTAs per SM on.  E4M3
-// caches take a shape of their own there (below; with fewer waves they keep four lanes of
-// three stages, with the 16-bit list).
+// units the coarser waves lose: the shape is used from five waves of three CTAs per SM on
+// (Hq 16, Hkv 2, W 2,051, S 65,536: 2,048 units 314 vs 306 us, 2,560 units 363 vs 381,
+// 3,072 units 432 vs 454).  E4M3 caches take a shape of their own there (below), from four
+// such waves on (2,048 units 227 vs 253 us, 1,280 units 191 vs 168); with fewer waves
+// they keep four lanes of three stages, with the 16-bit list.
 constexpr int64_t kRows16 = 65536;
 #ifndef QSA_SHAPE16_MIN_WAVES
-#define QSA_SHAPE16_MIN_WAVES 8
+#define QSA_SHAPE16_MIN_WAVES 5
+#endif
+#ifndef QSA_FP8_SHAPE16_MIN_WAVES
+#define QSA_FP8_SHAPE16_MIN_WAVES 4
 #endif
 constexpr int64_t kShape16MinWaves = QSA_SHAPE16_MIN_WAVES;
+constexpr int64_t kFp8Shape16MinWaves = QSA_FP8_SHAPE16_MIN_WAVES;
 #ifndef QSA_SMALL16_SL
 #define QSA_SMALL16_SL 2
 #endif
@@ -1208,15 +1213,16 @@ size_t workspace_bytes_for(int32_t Tq, int32_t Hq, int32_t nsplit) {
 }
 
 // Kernel shape of a call: by cache format and group size G; caches of at most 65,536 rows
-// take the 16-bit row list, and with it, in launches of at least eight waves, the shapes of
-// three CTAs per SM (G <= 8, and 8 < G <= 12 for bf16 caches).
+// take the 16-bit row list, and with it, in launches of at least five (E4M3: four) waves of
+// three CTAs per SM, the shapes of more resident CTAs (G <= 8, and 8 < G <= 12 for bf16
+// caches).
 cudaError_t launch_sparse_prefill(const FwdParams& p, cudaStream_t stream) {
   cudaError_t e;
   // every compacted row number is below the row count of this call's cache
   const bool rows16 = p.S <= kRows16;
   const int64_t grid = int64_t(p.Tq) * p.Hkv * p.nsplit;
-  const bool shape16 =
-      rows16 && p.num_sms > 0 && grid >= kShape16MinWaves * p.num_sms * 3;
+  const bool shape16 = rows16 && p.num_sms > 0 &&
+                       grid >= (p.kv_fp8 ? kFp8Shape16MinWaves : kShape16MinWaves) * p.num_sms * 3;
   // TMA tile::gather4 for the rows where it is the faster gather (per cache format; one
   // tensor map per KV head for K and V, so at most kMaxTmaHeads heads; an empty shard
   // (S == 0) gathers nothing and takes the cp.async kernel)

@@ -61,6 +61,42 @@ qsa_status_t qsa_probe_gather(int32_t method, int32_t read_back, const void* src
                               int32_t stages, int32_t ctas, int32_t iters, uint32_t seed,
                               uint32_t* sink, void* stream);
 
+/*
+ * qsa_probe_mma_operands -- enqueue one launch of the MMA operand-rate probe on `stream`.
+ *
+ * The fused kernel reads every gathered K and V row from shared memory once, into its
+ * matrix products.  On sm_100a that read can be done by the warps (ldmatrix into
+ * registers for the warp-level mma, the form the fused kernel uses) or by the tensor core
+ * itself (tcgen05.mma reads both operands through shared-memory matrix descriptors and
+ * accumulates in tensor memory).  This probe measures how many operand bytes per clock
+ * each form reads from one SM's shared memory, so the two can be compared at the skinny
+ * shapes of this path (many slots x a group of 8 to 16 heads).
+ *
+ *   method  0: ldmatrix.x4 by 16 warps over a 64 KiB window (n must be 0); bytes read per
+ *              CTA: rounds x 16 warps x 128 x 512.
+ *           1: tcgen05.mma.cta_group::1.kind::f16, M = 128, N = n, K = 16 per
+ *              instruction, bf16 K-major operands without swizzle, fp32 accumulator in
+ *              tensor memory, issued by one thread back to back, completion through
+ *              tcgen05.commit on an mbarrier (a bounded wait); bytes read per CTA:
+ *              rounds x 16 x (128 + n) x 32.  The operands are bf16 ones, so every
+ *              accumulator element must end at rounds x 256; each of the 128 lanes of column
+ *              0 is checked.
+ *   n       method 1: 16, 32, 64, 128 or 256.
+ *   rounds  1 .. 65,536 passes.
+ *   ctas    grid size (one CTA per SM is what the probe is sized for: the tcgen05 variant
+ *           takes 200 KiB of shared memory).
+ *   out     device int64 [2 + ctas], 8-byte aligned; the caller clears out[0] and out[1].
+ *           out[0] bit 0: a completion wait timed out (the launch is not a measurement);
+ *           out[1]: accumulator elements that are not rounds x 256 (method 1); out[2 + b]:
+ *           the SM clock cycles CTA b spent in its timed loop (clock64).
+ * Operand bytes per clock per SM = bytes read per CTA / max_b out[2 + b].  Returns
+ * QSA_ERR_INVALID_ARG for arguments outside the ranges above, QSA_ERR_CUDA if the launch
+ * fails.  Allocates nothing (the tensor memory the tcgen05 variant allocates is freed by
+ * the same CTA before it exits).
+ */
+qsa_status_t qsa_probe_mma_operands(int32_t method, int32_t n, int32_t rounds, int32_t ctas,
+                                    int64_t* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -351,6 +351,22 @@ def test_probe_valid_arguments_reach_the_device(lib):
     assert st == qsa.QSA_ERR_CUDA
 
 
+@pytest.mark.parametrize("over", [dict(method=2), dict(method=-1), dict(method=0, n=16),
+                                  dict(method=1, n=0), dict(method=1, n=48), dict(rounds=0),
+                                  dict(rounds=65537), dict(ctas=0), dict(out=0), dict(out=0x1004)])
+def test_mma_probe_rejects_bad_arguments_before_cuda(lib, over):
+    a = dict(method=1, n=16, rounds=10, ctas=4, out=0x1000)
+    a.update(over)
+    st = qsa.qsa_probe_mma_operands(a["method"], a["n"], a["rounds"], a["ctas"], a["out"], None)
+    assert st == qsa.QSA_ERR_INVALID_ARG, qsa.qsa_last_error_detail()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_mma_probe_valid_arguments_reach_the_device(lib):
+    assert qsa.qsa_probe_mma_operands(0, 0, 10, 4, 0x1000, None) == qsa.QSA_ERR_CUDA
+    assert qsa.qsa_probe_mma_operands(1, 256, 10, 4, 0x1000, None) == qsa.QSA_ERR_CUDA
+
+
 def test_partial_plan_workspace(lib):
     """A shard smaller than the cache with an unsplit plan asks for the compaction buffer
     ([Tq, W] and [Tq] int32, each 256-byte aligned); the whole cache, a narrow selection

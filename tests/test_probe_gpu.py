@@ -54,3 +54,18 @@ def test_gather_peak_is_plausible(cuda_device):
     assert all(x["tb_per_s"] is not None for x in r["runs"])
     assert r["tb_per_s"] == max(x["tb_per_s"] for x in r["runs"])
     assert 1.0 < r["tb_per_s"] < sms * 256 * 2.1e9 / 1e12
+
+
+def test_mma_operand_probe(cuda_device):
+    """The MMA operand-rate probe: every tcgen05 accumulator element comes out exact, no
+    wait times out, and the rates are positive; the tensor core's MAC rate at N = 256 is
+    the order of the dense peak (one MMA of 128 x 256 x 16 per ~128 cycles or better)."""
+    from top_sparse_attention_index_b200.gather_probe import MMA_N, mma_operand_rates
+    r = mma_operand_rates(cuda_device, rounds=200)
+    assert r["ldmatrix_x4_16_warps"]["timeouts"] == 0
+    assert r["ldmatrix_x4_16_warps"]["bytes_per_clk_per_sm"] > 0
+    for n in MMA_N:
+        d = r["tcgen05"][str(n)]
+        assert d["timeouts"] == 0 and d["mismatches"] == 0, (n, d)
+        assert d["bytes_per_clk_per_sm"] > 0
+    assert r["tcgen05"]["256"]["mac_per_clk_per_sm"] > 1000

@@ -25,6 +25,7 @@ from ._binding import (  # noqa: F401
     qsa_sparse_prefill_block,
     qsa_combine_partials,
     qsa_probe_gather,
+    qsa_probe_mma_operands,
     qsa_sparse_prefill_block_plan,
     qsa_sparse_prefill_fp8kv,
     qsa_sparse_prefill_partial,
@@ -54,5 +55,5 @@ __all__ = [
     "combine_partials", "sparse_prefill_context_parallel", "shard_ranges",
     "qsa_combine_peer_records", "combine_peer_records", "PeerExchange", "release_peer_exchanges",
     "qsa_sparse_prefill_plan", "qsa_sparse_prefill_workspace_bytes", "qsa_status_string", "qsa_last_error_detail", "qsa_abi_version",
-    "load_library", "QSAError", "qsa_probe_gather",
+    "load_library", "QSAError", "qsa_probe_gather", "qsa_probe_mma_operands",
 ]

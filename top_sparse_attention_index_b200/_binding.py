@@ -57,6 +57,7 @@ SIGNATURES = {
                                           _i64, _i64, _i32, _p, _p]),
     "qsa_probe_gather": (_i32, [_i32, _i32, _p, _i64, _i64, _i32, _i32, _i32, _i32, _i32,
                                 ctypes.c_uint32, _p, _p]),
+    "qsa_probe_mma_operands": (_i32, [_i32, _i32, _i32, _i32, _p, _p]),
     "qsa_combine_peer_records": (_i32, [ctypes.POINTER(_p), ctypes.POINTER(_p), _i32, _i32, _i32,
                                         _i32, _i32, _i32, _i32, ctypes.POINTER(_p), _i32, _i64,
                                         _i64, _p]),
@@ -135,6 +136,11 @@ def qsa_probe_gather(method, read_back, src, rows, pitch_bytes, row_bytes, warps
     return int(load_library().qsa_probe_gather(method, read_back, src, rows, pitch_bytes,
                                                row_bytes, warps_per_cta, stages, ctas, iters,
                                                seed, sink, stream))
+
+
+def qsa_probe_mma_operands(method, n, rounds, ctas, out, stream) -> int:
+    """Raw call of the MMA operand-rate probe (include/qsa_probe.h); returns the status."""
+    return int(load_library().qsa_probe_mma_operands(method, n, rounds, ctas, out, stream))
 
 
 def qsa_sparse_prefill(q, q_stride_t, q_stride_h, k_cache, k_stride_s, k_stride_h, v_cache,

@@ -19,7 +19,7 @@ CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 LIBRARY = PKG / "libqsa.so"
 SOURCES = [CSRC / "qsa_api.cu", CSRC / "qsa_attn.cu", CSRC / "qsa_noalloc.cu", CSRC / "qsa_probe.cu",
-           CSRC / "qsa_peer.cu"]
+           CSRC / "qsa_probe_mma.cu", CSRC / "qsa_peer.cu"]
 DEPENDS = SOURCES + [CSRC / "qsa_internal.h", CSRC / "qsa_ptx.cuh", INCLUDE / "qsa.h",
                      INCLUDE / "qsa_probe.h", INCLUDE / "qsa_peer.h"]
 

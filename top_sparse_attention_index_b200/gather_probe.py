@@ -11,10 +11,11 @@ shared memory, each landed row read back once with ldmatrix.  gather_peak() runs
 the loaders (the kernel's cp.async, and TMA tile::gather4) and a few pipeline shapes and
 returns the best rate; the benchmark reports the fused kernel against it.
 
-    python -m top_sparse_attention_index_b200.gather_probe [--rows 512|256] [--sweep]
+    python -m top_sparse_attention_index_b200.gather_probe [--rows 512|256] [--sweep] [--mma]
 
 prints one JSON line per run (--sweep: every method, with and without the read-back,
-over more shapes).  Needs a GPU; allocates a 64 MB buffer.
+over more shapes; --mma: the shared-memory operand rates of ldmatrix and tcgen05.mma,
+mma_operand_rates()).  Needs a GPU; allocates a 64 MB buffer.
 """
 from __future__ import annotations
 
@@ -130,14 +131,56 @@ def sweep(device, row_bytes: int, reps: int = 5):
                "timeouts": int(sink[0].item()), "layout_mismatches": int(sink[1].item())}
 
 
+MMA_N = (16, 32, 64, 128, 256)
+
+
+def mma_operand_rates(device, rounds: int = 2000) -> dict:
+    """Shared-memory operand bytes per clock per SM of the two MMA forms (the MMA probe of
+    include/qsa_probe.h, one CTA per SM): ldmatrix.x4 from 16 warps, and tcgen05.mma with
+    M = 128, K = 16 and N = 16 ... 256 (the accumulator checked exactly).  The gathered rows
+    are read from shared memory once whichever form reads them, so the faster reader at
+    this path's skinny shapes (many slots x 8-16 heads) is the one that can raise the
+    fused kernel's bound."""
+    from . import _binding as qsa
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    out = torch.zeros(2 + sms, dtype=torch.int64, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def run(method, n, bytes_per_cta):
+        for r in (1, rounds):  # a warm-up launch, then the measured one
+            out.zero_()
+            st = qsa.qsa_probe_mma_operands(method, n, r, sms, out.data_ptr(), stream.cuda_stream)
+            if st != qsa.QSA_OK:
+                raise qsa.QSAError(st, qsa.qsa_last_error_detail())
+        torch.cuda.synchronize(device)
+        o = out.cpu()
+        cycles = int(o[2:].max())
+        return {"timeouts": int(o[0]), "mismatches": int(o[1]), "cycles": cycles,
+                "bytes_per_clk_per_sm": bytes_per_cta(rounds) / cycles}
+
+    res = {"rounds": rounds, "ctas": sms,
+           "ldmatrix_x4_16_warps": run(0, 0, lambda r: r * 16 * 128 * 512), "tcgen05": {}}
+    for n in MMA_N:
+        d = run(1, n, lambda r, n=n: r * 16 * (128 + n) * 32)
+        mmas = rounds * 16
+        d.update({"M": 128, "N": n, "K": 16, "clk_per_mma": d["cycles"] / mmas,
+                  "mac_per_clk_per_sm": mmas * 128 * n * 16 / d["cycles"]})
+        res["tcgen05"][str(n)] = d
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--rows", type=int, choices=[512, 256], default=512,
                     help="row bytes: 512 (bf16, head dim 256) or 256 (E4M3 codes)")
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--mma", action="store_true",
+                    help="the MMA operand-rate probe instead (ldmatrix vs tcgen05.mma)")
     args = ap.parse_args()
     device = torch.device("cuda", 0)
-    if args.sweep:
+    if args.mma:
+        print(json.dumps(mma_operand_rates(device)))
+    elif args.sweep:
         for r in sweep(device, args.rows):
             print(json.dumps(r), flush=True)
     else:

@@ -253,3 +253,55 @@ def test_peer_exchange_protocol(oracle_lib):
                 assert np.abs(out - ref).max() <= bound
                 np.testing.assert_array_equal(out, results[0][0])
             assert np.all(results[r][0][1] == 0)   # the fully masked row
+
+
+# ---- a rank that fails: the others end with an error instead of waiting for good -------
+
+def _failing_rank_main(rank, world, port, queue, exchange):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    if rank == world - 1:
+        queue.put((rank, "left"))          # this rank leaves before the exchange
+        return
+    q, k, v, idx = _case()
+    S = k.shape[0]
+    lo, hi = cp.shard_ranges(S, world)[rank]
+    try:
+        kw = dict(partial_fn=_partial_into, peer_combine_fn=_peer_combine_emulated,
+                  ipc=_FakeIPC(rank)) if exchange == "peer" else \
+             dict(partial_fn=_partial_double, combine_fn=_combine_double)
+        cp.sparse_prefill_context_parallel(q, k[lo:hi], v[lo:hi], idx, lo, S, exchange=exchange,
+                                           record_dtype=torch.float32, **kw)
+        queue.put((rank, "no error"))
+    except Exception as e:  # noqa: BLE001 - the collective's error is what the test wants
+        queue.put((rank, "error: " + type(e).__name__))
+
+
+def test_a_rank_that_leaves_ends_the_exchange_with_an_error():
+    """World size 3 with a 5-second process-group timeout; the last rank leaves before the
+    exchange (host-side failure, no device involved).  The remaining ranks' exchange (the
+    all-gather, or the peer exchange's handle exchange and barriers) ends with an error
+    within the timeout instead of waiting for good."""
+    import time
+    for exchange in ("all_gather", "peer"):
+        ctx = mp.get_context("spawn")
+        queue = ctx.Queue()
+        port = _free_port()
+        procs = [ctx.Process(target=_failing_rank_main, args=(r, 3, port, queue, exchange))
+                 for r in range(3)]
+        t0 = time.time()
+        for p in procs:
+            p.start()
+        results = dict(queue.get(timeout=120) for _ in procs)
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+                p.join()
+        assert results[2] == "left"
+        for r in (0, 1):
+            assert results[r].startswith("error"), (exchange, results)
+        assert time.time() - t0 < 110

@@ -741,8 +741,8 @@ def test_context_parallel_block4_and_empty_shard(cuda_device, oracle_lib):
 
 def test_context_parallel_nccl_world_of_one(cuda_device):
     """The public context-parallel call end to end on one GPU: a one-rank NCCL group,
-    its all-gather and the combine; one shard holding the whole cache gives bitwise the
-    unsharded call."""
+    its all-gather and the combine, then the peer exchange with its NCCL barriers; one
+    shard holding the whole cache gives bitwise the unsharded call either way."""
     import datetime
     import os
     import socket
@@ -764,6 +764,16 @@ def test_context_parallel_nccl_world_of_one(cuda_device):
         out = qsa.sparse_prefill_context_parallel(d["q"], d["k_cache"][lo:hi], d["v_cache"][lo:hi],
                                                   d["slot_idx"], lo, w.S, width=d["width"])
         torch.cuda.synchronize()
-        assert torch.equal(out.cpu().view(torch.int16), run(d, 1.0 / 16.0).view(torch.int16))
+        unsharded = run(d, 1.0 / 16.0).view(torch.int16)
+        assert torch.equal(out.cpu().view(torch.int16), unsharded)
+        # the peer exchange over the same group: its buffers, the NCCL barriers on the
+        # compute stream and the combine of this rank's rows (all of them), twice
+        for _ in range(2):
+            out = qsa.sparse_prefill_context_parallel(d["q"], d["k_cache"][lo:hi], d["v_cache"][lo:hi],
+                                                      d["slot_idx"], lo, w.S, width=d["width"],
+                                                      exchange="peer")
+            torch.cuda.synchronize()
+            assert torch.equal(out.cpu().view(torch.int16), unsharded)
+        qsa.release_peer_exchanges()
     finally:
         dist.destroy_process_group()

@@ -45,6 +45,11 @@ __global__ void __launch_bounds__(128)
   const int64_t row = int64_t(p.t0) * p.Hq + i;  // (t, h) row of the records
   const int64_t t = row / p.Hq, h = row % p.Hq;
   const float lse_l = lane < p.R ? p.rec_lse[lane][row] : kNegInfP;
+  // lane r holds record r's row address; the loop takes it with a shuffle
+  const unsigned long long o_l =
+      lane < p.R ? reinterpret_cast<unsigned long long>(p.rec_o[lane]) +
+                       static_cast<unsigned long long>(row) * qsa::kHeadDim * (IN_BF16 ? 2 : 4)
+                 : 0ull;
   float mstar = lse_l;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mstar = fmaxf(mstar, __shfl_xor_sync(0xffffffffu, mstar, off));
@@ -60,16 +65,16 @@ __global__ void __launch_bounds__(128)
 #pragma unroll kPeerUnroll
     for (int r = 0; r < p.R; ++r) {
       const float lse = __shfl_sync(0xffffffffu, lse_l, r);
-      const int64_t off = row * qsa::kHeadDim + lane * 8;
+      const unsigned long long rowp = __shfl_sync(0xffffffffu, o_l, r);
       float x[8];
       if constexpr (IN_BF16) {
-        const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.rec_o[r]) + off);
+        const uint4 v = *(reinterpret_cast<const uint4*>(rowp) + lane);
         x[0] = bf16lo_to_f32(v.x); x[1] = bf16hi_to_f32(v.x);
         x[2] = bf16lo_to_f32(v.y); x[3] = bf16hi_to_f32(v.y);
         x[4] = bf16lo_to_f32(v.z); x[5] = bf16hi_to_f32(v.z);
         x[6] = bf16lo_to_f32(v.w); x[7] = bf16hi_to_f32(v.w);
       } else {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.rec_o[r]) + off);
+        const float4* src = reinterpret_cast<const float4*>(rowp) + 2 * lane;
         const float4 a = src[0], b = src[1];
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
         x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;

@@ -383,3 +383,39 @@ def test_partial_plan_workspace(lib):
         with pytest.raises(qsa.QSAError) as ei:
             qsa.qsa_sparse_prefill_partial_plan(4, 16, 2, 256, 64, 1, S, S_total, 148)
         assert ei.value.status == qsa.QSA_ERR_INVALID_ARG
+
+
+def test_plan_properties_on_random_shapes(lib):
+    """Seeded random shapes through the planner (host only): every split holds at most
+    2,240 slots (the per-split slot list in shared memory), no split lies wholly past W,
+    a split is never narrower than 128 slots unless W itself forces it, batches of at
+    least one wave of units are not split beyond what W forces, a forced request is
+    honoured within those limits, and the workspace is the fp32 partials plus the LSEs,
+    each region 256-byte aligned (none without a split)."""
+    import random
+    rng = random.Random(2024)
+    max_slots, min_slots, wave = 2240, 128, 148 * 2
+    for _ in range(3000):
+        Hkv = rng.choice([1, 2, 3, 4, 8])
+        Hq = Hkv * rng.randint(1, 16)
+        Tq = rng.choice([rng.randint(1, 16), rng.randint(1, 400), rng.randint(1, 20000)])
+        block = rng.choice([1, 1, 1, 2, 4, 16])
+        W = rng.randint(1, 30000 // block)
+        request = rng.choice([0, 0, rng.randint(1, 64)])
+        n, ws = qsa.qsa_sparse_prefill_block_plan(Tq, Hq, Hkv, 256, W, block, 148, request)
+        per_split = -(-W // n)                        # entries per split
+        min_split = -(-W * block // max_slots)
+        assert 1 <= n <= W and per_split * block <= max_slots, (Tq, Hq, Hkv, W, block, n)
+        assert (n - 1) * per_split < W, "a split lies wholly past W"
+        # the count the plan settles on for a wanted count (no split wholly past W)
+        settle = lambda k: -(-W // -(-W // k))  # noqa: E731
+        if request == 0:
+            if Tq * Hkv >= wave:
+                assert n == settle(min_split), (Tq, Hkv, W, n)
+            elif n > settle(min_split):
+                assert per_split * block >= min_slots, (Tq, Hkv, W, block, n)
+        else:
+            assert n == settle(min(max(request, min_split), W)), (W, block, request, n)
+        r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+        want = 0 if n == 1 else r256(n * Tq * Hq * 256 * 4) + r256(n * Tq * Hq * 4)
+        assert ws == want, (Tq, Hq, Hkv, W, block, n, ws, want)
